@@ -1,0 +1,340 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid-attention forward (one layer call = one step).
+
+Default workload: the Wan-2.1-1.3B-shaped bidirectional layer (B=1, H=12,
+d=128, 21 frames x 1560 tokens, 3-frame chunks +/- 1 frame, bf16). Prints one
+JSON line: effective TFLOP/s (kept-window pairs x 4d plus linear-state FLOPs)
+over all ranks, tokens/s, the dominant kernel's roofline, the oracle's CPU
+throughput on a bounded sample, an end-to-end figure through the public API
+with host buffers, and the SM clocks seen during the timed region.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload NAME]
+
+Multi-GPU: one process per GPU (torchrun). Batch elements are independent, so
+each rank runs its own layer call on its own inputs (weak scaling, no
+data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_video_hyat_b200 import workloads as wl  # noqa: E402
+
+METRIC = "hybrid-attn effective TFLOP/s & tokens/s per layer; % of B200 BF16 TC peak"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["linear_attention_video_hyat_b200/csrc/attn_tc.cu"]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=wl.WAN13B_BIDIR.name, choices=sorted(wl.WORKLOADS))
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- work counts
+def work_counts(w):
+    """Effective FLOPs of one call and the attention kernel's share, from the library layout."""
+    from linear_attention_video_hyat_b200 import hyat
+    cfg = hyat.config_from_workload(w)
+    work, ent = hyat.plan_layout(cfg)
+    per_bh = work[work[:, 0] == 0]
+    klen = np.concatenate([[0], np.cumsum(ent[:, 1].astype(np.int64))])
+    pairs = int(sum(int(it[2]) * int(klen[it[5]] - klen[it[4]]) for it in per_bh))
+    BH, d, N = w.B * w.H, w.d, w.N
+    soft = 4 * d * pairs * BH
+    fold = BH * N * (2 * d * d + d)
+    apply = BH * N * (2 * d * d + 2 * d)
+    return {"pairs_per_head": pairs, "softmax_flops": soft, "state_flops": fold + apply,
+            "total_flops": soft + fold + apply, "attn_kernel_flops": soft + apply,
+            "state_kernel_bytes": 2 * BH * N * d * 2 + BH * (N // w.tokens_per_frame) * (d * d + d) * 4}
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the GPU runs."""
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+        self.names = {}
+        if self._ok:
+            for name in ("HwSlowdown", "HwThermalSlowdown", "SwThermalSlowdown", "SwPowerCap", "HwPowerBrakeSlowdown"):
+                for prefix in ("nvmlClocksEventReason", "nvmlClocksThrottleReason"):
+                    v = getattr(self.nv, prefix + name, None)
+                    if v is not None:
+                        self.names[name] = v
+                        break
+
+    def _run(self):
+        get_reasons = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = get_reasons(self.h)
+                for n, bit in self.names.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self.t.join()
+
+    def summary(self):
+        snake = {"HwSlowdown": "hw_slowdown", "HwThermalSlowdown": "hw_thermal_slowdown",
+                 "SwThermalSlowdown": "sw_thermal_slowdown", "SwPowerCap": "sw_power_cap",
+                 "HwPowerBrakeSlowdown": "hw_power_brake_slowdown"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": sorted(snake[r] for r in self.reasons)}
+
+
+# ----------------------------------------------------------------- oracle (CPU) leg
+def oracle_sample(w, n_blocks, rows_per_block=256, seed=0, qkv=None):
+    """Time the fp64 oracle on `n_blocks` blocks of query rows; returns (seconds, rows)."""
+    import oracle
+    q, k, v = wl.gen_qkv(w) if qkv is None else qkv
+    rng = np.random.default_rng(seed)
+    t = 0.0
+    rows_done = 0
+    for b in range(n_blocks):
+        h = int(rng.integers(0, w.H))
+        r0 = int(rng.integers(0, w.N - rows_per_block + 1))
+        rows = np.arange(r0, r0 + rows_per_block)
+        qs = q[:, h:h + 1].float().numpy()
+        ks = k[:, h:h + 1].float().numpy()
+        vs = v[:, h:h + 1].float().numpy()
+        t0 = time.perf_counter()
+        if w.mode == "window":
+            oracle.bidir_window_attention(qs, ks, vs, w.tokens_per_frame, w.n_frames, w.chunk_frames,
+                                          w.halo_frames, rows=rows)
+        elif w.mode == "radial":
+            oracle.radial_attention(qs, ks, vs, w.n_frames, w.tokens_per_frame, rows=rows)
+        else:
+            raise ValueError("oracle timing covers the bidirectional workloads")
+        t += time.perf_counter() - t0
+        rows_done += rows_per_block
+    return t, rows_done
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_rate(w, counts, n_blocks, qkv=None):
+    secs, rows = oracle_sample(w, n_blocks, qkv=qkv)
+    total_rows = w.B * w.H * w.N
+    frac = rows / total_rows
+    tflops = counts["total_flops"] * frac / secs / 1e12
+    return tflops, rows / secs, secs, rows
+
+
+# ----------------------------------------------------------------- main
+def main():
+    a = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    w = wl.WORKLOADS[a.workload]
+    assert w.mode in ("window", "radial"), "the bench times a bidirectional layer call"
+    counts = work_counts(w)
+    config = {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "tokens": w.N,
+              "tokens_per_frame": w.tokens_per_frame, "frames": w.n_frames, "mode": w.mode,
+              "chunk_frames": w.chunk_frames, "halo_frames": w.halo_frames,
+              "parallelism": f"replicas{world}" if world > 1 else "single",
+              "l2": "inputs larger than L2 (Q,K,V,O %.0f MB > 126 MB); no flush" % (4 * w.B * w.H * w.N * w.d * 2 / 1e6)}
+
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        qkv = wl.gen_qkv(w)
+        for _ in range(a.warmup):
+            oracle_sample(w, 1, seed=99, qkv=qkv)
+        secs, rows = 0.0, 0
+        for i in range(a.steps):
+            s, r = oracle_sample(w, 1, seed=i, qkv=qkv)
+            secs += s
+            rows += r
+        frac = rows / (w.B * w.H * w.N)
+        value = counts["total_flops"] * frac / secs / 1e12
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": 1e3 * secs / a.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "impl": "reference", "tokens_per_s": rows / secs,
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                                 "sample": f"{a.steps} blocks of 256 query rows (one head each) per run"},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    from linear_attention_video_hyat_b200 import hyat
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    q, k, v = wl.gen_qkv(w, seed=w.seed + rank)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    od = torch.empty_like(qd)
+    h = hyat.Hyat(hyat.config_from_workload(w), device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(a.warmup, 3)):
+        h.forward(qd, kd, vd, out=od)
+    h.sync()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+
+    h.set_profiling(True)
+    h.kernel_times()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for _ in range(a.steps):
+            h.forward(qd, kd, vd, out=od)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    h.sync()
+    ms = t0.elapsed_time(t1) / a.steps
+    kt = h.kernel_times()
+    h.set_profiling(False)
+    if world > 1:
+        mt = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(mt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(mt.item())
+    launches = sum(n for _, n in kt.values())
+
+    value = counts["total_flops"] * world / (ms / 1e3) / 1e12
+    tokens_per_s = w.B * w.N * world / (ms / 1e3)
+    pk, pk_src = peaks()
+    attn_ms = kt["attention"][0] / max(kt["attention"][1], 1)
+    achieved = counts["attn_kernel_flops"] / (attn_ms / 1e3) / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if os.path.exists(tpath):
+        t = json.load(open(tpath))
+        sha = hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read() for f in KERNEL_SOURCES)).hexdigest()
+        if t.get("source_sha256") == sha and t.get("workload") == w.name:
+            traffic = t.get("dram_bytes_per_launch")
+    roofline = {"bound": "tensor", "kernel": "attention", "achieved": achieved,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                "peak_kind": f"{pk_src} bf16 burst", "peak_sustained": pk["bf16_tflops_sustained"],
+                "frac_sustained": achieved / pk["bf16_tflops_sustained"], "traffic": traffic,
+                "launch_ms": attn_ms, "algorithmic_flops_per_launch": counts["attn_kernel_flops"]}
+    kernels = {k_: {"ms_per_launch": t_ / max(n_, 1), "launches": n_} for k_, (t_, n_) in kt.items() if n_}
+    state_ms = kernels.get("state", {}).get("ms_per_launch")
+    if state_ms:
+        kernels["state"]["hbm_gbs"] = counts["state_kernel_bytes"] / (state_ms / 1e3) / 1e9
+
+    e2e = None
+    if not a.no_e2e:
+        qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+        oh = torch.empty_like(qh).pin_memory()
+        e_steps = max(3, min(a.steps, 20))
+        for _ in range(2):
+            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+            h.forward(qd, kd, vd, out=od)
+            oh.copy_(od, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+            h.forward(qd, kd, vd, out=od)
+            oh.copy_(od, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = e0.elapsed_time(e1) / e_steps
+        if world > 1:
+            mt = torch.tensor([ems], device=dev)
+            torch.distributed.all_reduce(mt, op=torch.distributed.ReduceOp.MAX)
+            ems = float(mt.item())
+        e2e = {"value": counts["total_flops"] * world / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": ems, "tokens_per_s": w.B * w.N * world / (ems / 1e3),
+               "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+               "d2h_bytes_per_step": q.numel() * q.element_size()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        tf, rps, secs, rows = cpu_rate(w, counts, n_blocks=24, qkv=(q, k, v))
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+               "tokens_per_s": rps, "seconds": secs,
+               "sample": f"{rows} query rows (24 blocks of 256 rows, one head each) of the same layer; "
+                         f"FLOPs scaled by the sampled fraction of rows"}
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+                "tokens_per_s": tokens_per_s, "frac_of_peak": value / world / pk["bf16_tflops"],
+                "effective_flops_per_step": counts["total_flops"] * world,
+                "roofline": roofline, "kernels": kernels, "gpu_launches": launches,
+                "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

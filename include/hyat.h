@@ -1,0 +1,184 @@
+/*
+ * hyat.h -- C interface of libhyat, hybrid softmax-window + linear-state
+ * attention (forward) for video diffusion transformers on NVIDIA B200 (sm_100a).
+ *
+ * The operation (ReHyAt: Recurrent Hybrid Attention for Video Diffusion
+ * Transformers, Abstract; Long-Horizon Streaming Video Generation via Hybrid
+ * Attention with Decoupled Distillation, Section 2.A "Hybrid Attention";
+ * Radial Attention: O(n log n) Sparse Attention with Energy Decay for Long
+ * Video Generation, Abstract): each query i takes exact softmax attention over
+ * the keys of its window W_i and reaches every other key j in its linear set
+ * R_i through the linear-attention state S = sum phi(k_j) v_j^T, z = sum phi(k_j),
+ * under one normaliser:
+ *
+ *   o_i = ( sum_{j in W_i} e^{s_ij - m_i} v_j + e^{-m_i} phi(q_i)^T S )
+ *       / ( sum_{j in W_i} e^{s_ij - m_i}     + e^{-m_i} phi(q_i)^T z ),
+ *   s_ij = scale * q_i . k_j,   phi(x) = elu(x) + 1,   m_i = max(0, max_j s_ij).
+ *
+ * Modes (hyat_config.mode):
+ *   WINDOW     bidirectional; frames of tokens_per_frame tokens are grouped in
+ *              chunks of chunk_frames; a query's window is its chunk plus
+ *              halo_frames frames on each side, clipped to the video; R_i is
+ *              every other token (token-exact).
+ *   BLOCKMASK  bidirectional; W_i is the union of the 128x128 tiles that a
+ *              caller mask keeps on the absolute tile grid; R_i is the rest.
+ *   RADIAL     BLOCKMASK with the static radial mask built by the library: a
+ *              tile is kept iff it holds a near pair (same frame, or
+ *              2*|p_j - p_i| < tokens_per_frame >> floor(log2 t) at frame
+ *              distance t, p = raster index inside the frame).
+ *   STREAM     causal streaming in chunks of chunk_frames frames; the KV window
+ *              holds the latest window_frames frames (a multiple of
+ *              chunk_frames); chunks that leave the window are folded into the
+ *              recurrent state (S, z); queries of the current chunk attend to
+ *              the kept 128x128 tiles of the window (per-step mask) and to the
+ *              state. Dropped window tiles reach neither branch.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors Q, K, V, O are row-major [B, H, N, d] (N = tokens), contiguous,
+ *     device memory, 16-byte aligned, dtype = hyat_config.dtype. O has Q's
+ *     shape. The caller owns them.
+ *   - The workspace is device memory owned by the caller, at least
+ *     hyat_workspace_bytes() bytes, 256-byte aligned, untouched by the caller
+ *     while the handle lives. The library never calls cudaMalloc on a
+ *     forward call.
+ *   - Every forward call is enqueued on the given stream (a cudaStream_t
+ *     passed as void*; NULL = legacy default stream) and returns without
+ *     waiting for the GPU. A device-side timeout (a bounded wait that gave up)
+ *     sets a status word in the workspace; hyat_sync() reports it as
+ *     HYAT_ERR_DEVICE_TIMEOUT.
+ *   - Nothing aborts or prints. Every failure returns a status; the text of
+ *     the last failure on a handle is hyat_last_error(handle).
+ *   - A handle is not thread-safe. Different handles are independent.
+ */
+#ifndef HYAT_H_
+#define HYAT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HYAT_API __attribute__((visibility("default")))
+#else
+#define HYAT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HYAT_OK = 0,
+  HYAT_ERR_INVALID_ARG = 1,     /* bad shape, pointer, alignment, mask or call order */
+  HYAT_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. d not in {64,128}) */
+  HYAT_ERR_CUDA = 3,            /* a CUDA runtime call failed; see hyat_last_error */
+  HYAT_ERR_DEVICE_TIMEOUT = 4,  /* a device-side bounded wait gave up */
+  HYAT_ERR_STATE = 5            /* stream state blob malformed or mismatched */
+} hyat_status;
+
+typedef enum { HYAT_F32 = 0, HYAT_BF16 = 1 } hyat_dtype;
+typedef enum { HYAT_PHI_ELU1 = 0 } hyat_phi;
+typedef enum {
+  HYAT_MODE_WINDOW = 0,
+  HYAT_MODE_BLOCKMASK = 1,
+  HYAT_MODE_RADIAL = 2,
+  HYAT_MODE_STREAM = 3
+} hyat_mode;
+
+/* Flags (hyat_config.flags). */
+#define HYAT_FLAG_SIMT 1u        /* run bf16 through the CUDA-core path (cross-check) */
+
+typedef struct {
+  int32_t B, H, d;               /* d in {64, 128} */
+  int32_t tokens_per_frame;      /* F */
+  int32_t n_frames;              /* T (bidirectional modes); ignored by STREAM */
+  int32_t chunk_frames;          /* WINDOW: chunk; STREAM: frames per step */
+  int32_t halo_frames;           /* WINDOW: frames added on each side of a chunk */
+  int32_t window_frames;         /* STREAM: frames kept in the KV window */
+  int32_t mode;                  /* hyat_mode */
+  int32_t dtype;                 /* hyat_dtype */
+  int32_t phi;                   /* hyat_phi */
+  int32_t mask_heads;            /* BLOCKMASK / STREAM masks: 1 (shared) or H */
+  uint32_t flags;                /* HYAT_FLAG_* */
+  float scale;                   /* softmax logit scale; 0 => 1/sqrt(d) */
+} hyat_config;
+
+typedef struct hyat_ctx* hyat_handle;
+
+/* Bytes of device workspace a handle of this configuration needs (an upper
+ * bound independent of the mask). Returns 0 if the configuration is invalid. */
+HYAT_API size_t hyat_workspace_bytes(const hyat_config* cfg);
+
+/* Create a handle. `host_mask` is read only by BLOCKMASK: uint8
+ * [mask_heads, nT, nT], nT = ceil(N/128), nonzero = tile kept; NULL elsewhere.
+ * Builds the layout on the host (and the radial mask for RADIAL), copies it
+ * into the workspace (synchronously, on the legacy stream) and zeroes the
+ * stream state. On failure *out is NULL. */
+HYAT_API hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspace_bytes,
+                                 const uint8_t* host_mask, hyat_handle* out);
+
+/* Bidirectional forward (WINDOW, BLOCKMASK, RADIAL): O = hybrid(Q, K, V).
+ * Q, K, V, O: [B, H, T*F, d] device pointers. Enqueues the state kernel, the
+ * complement reduction and the attention kernel on `stream`. */
+HYAT_API hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const void* v,
+                           void* o, void* stream);
+
+/* One streaming step (STREAM): Q, K, V, O are the current chunk,
+ * [B, H, L, d], L = chunk_frames * F. `host_step_mask` is uint8
+ * [mask_heads, nQT, nQT * nwin] on the host (nQT = ceil(L/128), nwin = number
+ * of window chunks visible at this step = min(step + 1, window_frames /
+ * chunk_frames), key tiles ordered oldest chunk first), or NULL for all tiles
+ * kept. Its diagonal tiles of the newest chunk must be set. Steps run in order;
+ * the step counter lives in the handle. Before attention, the chunk leaving
+ * the window (if any) is folded into S, z and the new K, V enter its ring slot. */
+HYAT_API hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, const void* v,
+                                 void* o, const uint8_t* host_step_mask, void* stream);
+
+/* Wait for the last call's stream and report device-side errors. */
+HYAT_API hyat_status hyat_sync(hyat_handle h);
+
+/* Release a handle (does not free the caller's workspace). NULL is accepted. */
+HYAT_API hyat_status hyat_destroy(hyat_handle h);
+
+HYAT_API const char* hyat_last_error(hyat_handle h);
+HYAT_API const char* hyat_status_string(hyat_status s);
+
+/* ---- inspection and test hooks (host-only unless stated) ---- */
+
+/* Host-only layout of a bidirectional configuration, without a GPU.
+ * Work items are 8 int32 each: {bh, q_row, q_len, state_group, entry_begin,
+ * entry_end, 0, 0}; entries are 2 int32 each: {k_row, k_len}. Counts are
+ * written to counts[0] (work items) and counts[1] (entries); if a capacity is
+ * too small the arrays are not written and HYAT_ERR_INVALID_ARG returned. */
+HYAT_API hyat_status hyat_plan_layout(const hyat_config* cfg, const uint8_t* host_mask,
+                             int32_t* work, size_t work_cap, int32_t* entries,
+                             size_t entries_cap, int64_t* counts);
+
+/* Host-only radial tile mask: out = uint8 [nT, nT], nT = ceil(T*F/128). */
+HYAT_API hyat_status hyat_radial_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t* out,
+                             size_t out_bytes);
+
+/* Host-only streaming bookkeeping of step `step`: info[0] = first visible
+ * chunk, info[1] = number of visible chunks, info[2] = chunk folded into the
+ * state before this step's attention (-1 if none), info[3] = ring slot
+ * receiving this step's K/V, info[4 + w] = ring slot of visible chunk w. */
+HYAT_API hyat_status hyat_stream_plan(const hyat_config* cfg, int32_t step, int32_t* info,
+                             size_t info_len);
+
+/* Stream state (S, z, KV ring, step) to / from a host buffer. The size is
+ * hyat_stream_state_bytes(); both calls synchronise the device. */
+HYAT_API size_t hyat_stream_state_bytes(hyat_handle h);
+HYAT_API hyat_status hyat_stream_get_state(hyat_handle h, void* dst_host, size_t bytes);
+HYAT_API hyat_status hyat_stream_set_state(hyat_handle h, const void* src_host, size_t bytes);
+
+/* Kernel timing: when enabled, each forward call records CUDA events around
+ * its launches; hyat_kernel_times() returns the summed milliseconds and
+ * launch counts per kernel kind since the last reset (kinds: 0 state,
+ * 1 complement, 2 attention, 3 stream fold + ring copy, 4 layout/prep).
+ * Reading the times synchronises the device. */
+HYAT_API hyat_status hyat_set_profiling(hyat_handle h, int enable);
+HYAT_API hyat_status hyat_kernel_times(hyat_handle h, double* ms, int64_t* launches, int n_kinds);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYAT_H_ */

@@ -1,0 +1,535 @@
+// C ABI of libhyat: handles, workspace planning, argument validation and
+// launch sequencing on the caller's stream.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "hyat_internal.h"
+
+using namespace hyat;
+
+namespace {
+
+constexpr int kKinds = 5;  // state, complement, attention, fold+ring, layout/prep
+enum Kind { K_STATE = 0, K_COMPLEMENT = 1, K_ATTN = 2, K_FOLD = 3, K_PREP = 4 };
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Plan {
+  size_t status = 0, work = 0, entries = 0, cm = 0, sseg = 0, srest = 0, srest_t = 0;
+  size_t ring_k = 0, ring_v = 0, mask = 0, total = 0;
+  int64_t n_work = 0, n_entries = 0;
+};
+
+int64_t elem_bytes(const hyat_config& c) { return c.dtype == HYAT_F32 ? 4 : 2; }
+
+// Offsets of every region in the caller's workspace.
+Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const Layout& L) {
+  Plan p;
+  const int64_t BH = int64_t(c.B) * c.H;
+  const int64_t E = int64_t(c.d) * c.d + c.d;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 256); return o; };
+  p.n_work = n_work;
+  p.n_entries = n_entries;
+  p.status = take(256);
+  p.work = take(sizeof(WorkItem) * std::max<int64_t>(n_work, 1));
+  p.entries = take(sizeof(Entry) * std::max<int64_t>(n_entries, 1));
+  if (c.mode == HYAT_MODE_STREAM) {
+    const int64_t Lc = stream_chunk_tokens(c), nwc = stream_window_chunks(c), nqt = tiles(Lc);
+    p.srest = take(sizeof(float) * BH * E);
+    p.srest_t = take(2 * BH * c.d * c.d);
+    p.ring_k = take(size_t(BH * nwc * Lc * c.d * elem_bytes(c)));
+    p.ring_v = take(size_t(BH * nwc * Lc * c.d * elem_bytes(c)));
+    p.mask = take(size_t(c.mask_heads) * nqt * nqt * nwc);
+  } else {
+    p.cm = take(sizeof(float) * size_t(L.cm_heads) * L.nqg * L.nseg);
+    p.sseg = take(sizeof(float) * BH * L.nseg * E);
+    p.srest = take(sizeof(float) * BH * L.nqg * E);
+    p.srest_t = take(2 * BH * L.nqg * c.d * c.d);
+  }
+  p.total = off;
+  return p;
+}
+
+// Counts of work items and entries (exact, or an upper bound for BLOCKMASK without a mask).
+bool plan_counts(const hyat_config& c, const uint8_t* host_mask, Layout* L, int64_t* n_work,
+                 int64_t* n_entries, std::string* err) {
+  if (c.mode == HYAT_MODE_STREAM) {
+    *err = build_layout(c, nullptr, L);
+    const int64_t nqt = tiles(stream_chunk_tokens(c));
+    *n_work = int64_t(c.B) * c.H * nqt;
+    *n_entries = *n_work * nqt * stream_window_chunks(c);
+    return err->empty();
+  }
+  if (c.mode == HYAT_MODE_BLOCKMASK && host_mask == nullptr) {
+    const int64_t nT = tiles(rows_q(c));
+    L->nseg = static_cast<int32_t>(nT);
+    L->nqg = static_cast<int32_t>(nT);
+    L->cm_heads = c.mask_heads;
+    *n_work = int64_t(c.B) * c.H * nT;
+    *n_entries = int64_t(c.mask_heads) * nT * nT;
+    return true;
+  }
+  *err = build_layout(c, host_mask, L);
+  if (!err->empty()) return false;
+  *n_work = static_cast<int64_t>(L->work.size());
+  *n_entries = static_cast<int64_t>(L->entries.size());
+  return true;
+}
+
+}  // namespace
+
+struct hyat_ctx {
+  hyat_config cfg{};
+  Layout lay;
+  Plan plan;
+  int32_t BH = 0, E = 0;
+  int64_t rq = 0, rk = 0;
+  char* ws = nullptr;
+  uint32_t* d_status = nullptr;
+  WorkItem* d_work = nullptr;
+  Entry* d_entries = nullptr;
+  float* d_cm = nullptr;
+  float* d_sseg = nullptr;
+  float* d_srest = nullptr;
+  uint16_t* d_srest_t = nullptr;
+  void* d_ring_k = nullptr;
+  void* d_ring_v = nullptr;
+  uint8_t* d_mask = nullptr;
+  int32_t step = 0;
+  bool use_tc = false;
+  int num_sms = 148;
+  cudaStream_t last_stream = nullptr;
+  std::string err;
+  bool profiling = false;
+  struct Rec { int kind; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> free_events;
+  double ms[kKinds] = {};
+  int64_t launches[kKinds] = {};
+};
+
+namespace {
+
+hyat_status fail(hyat_ctx* h, hyat_status s, const std::string& msg) {
+  if (h) h->err = msg;
+  return s;
+}
+
+hyat_status cuda_fail(hyat_ctx* h, cudaError_t e, const char* what) {
+  return fail(h, HYAT_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+cudaEvent_t get_event(hyat_ctx* h) {
+  if (!h->free_events.empty()) {
+    cudaEvent_t e = h->free_events.back();
+    h->free_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Times the launches issued by `fn` when profiling is on.
+template <typename Fn>
+cudaError_t timed(hyat_ctx* h, int kind, cudaStream_t s, Fn&& fn) {
+  if (!h->profiling) return fn();
+  cudaEvent_t a = get_event(h), b = get_event(h);
+  if (a) cudaEventRecord(a, s);
+  cudaError_t e = fn();
+  if (b) cudaEventRecord(b, s);
+  if (a && b) h->recs.push_back({kind, a, b});
+  return e;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hyat_status check_ptrs(hyat_ctx* h, const void* q, const void* k, const void* v, const void* o) {
+  if (!q || !k || !v || !o) return fail(h, HYAT_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(h, HYAT_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  return HYAT_OK;
+}
+
+AttnArgs attn_args(hyat_ctx* h, const void* q, const void* k, const void* v, void* o, int64_t n_work,
+                   int32_t nqg) {
+  AttnArgs a{};
+  a.q = q; a.k = k; a.v = v; a.o = o;
+  a.q_rows = h->rq;
+  a.k_rows = h->rk;
+  a.work = h->d_work;
+  a.n_work = static_cast<int32_t>(n_work);
+  a.entries = h->d_entries;
+  a.srest = h->d_srest;
+  a.srest_t = h->d_srest_t;
+  a.nqg = nqg;
+  a.d = h->cfg.d;
+  a.dtype = h->cfg.dtype;
+  a.BH = h->BH;
+  const float scale = h->cfg.scale > 0.0f ? h->cfg.scale : 1.0f / std::sqrt(float(h->cfg.d));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.status = h->d_status;
+  return a;
+}
+
+hyat_status launch_attention(hyat_ctx* h, const AttnArgs& a, cudaStream_t s) {
+  cudaError_t e;
+  if (h->use_tc) {
+    e = timed(h, K_PREP, s, [&] {
+      return launch_state_transpose_bf16(h->d_srest, h->d_srest_t, int64_t(h->BH) * a.nqg, h->cfg.d, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(h, e, "state transpose");
+    e = timed(h, K_ATTN, s, [&] { return launch_attn_tc(a, h->num_sms, s); });
+  } else {
+    e = timed(h, K_ATTN, s, [&] { return launch_attn_simt(a, s); });
+  }
+  if (e != cudaSuccess) return cuda_fail(h, e, "attention kernel");
+  return HYAT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hyat_status_string(hyat_status s) {
+  switch (s) {
+    case HYAT_OK: return "ok";
+    case HYAT_ERR_INVALID_ARG: return "invalid argument";
+    case HYAT_ERR_UNSUPPORTED: return "unsupported";
+    case HYAT_ERR_CUDA: return "CUDA error";
+    case HYAT_ERR_DEVICE_TIMEOUT: return "device timeout";
+    case HYAT_ERR_STATE: return "bad stream state";
+  }
+  return "unknown status";
+}
+
+const char* hyat_last_error(hyat_handle h) { return h ? h->err.c_str() : "null handle"; }
+
+size_t hyat_workspace_bytes(const hyat_config* cfg) {
+  if (!cfg || !validate_config(*cfg).empty()) return 0;
+  Layout L;
+  int64_t nw = 0, ne = 0;
+  std::string err;
+  if (!plan_counts(*cfg, nullptr, &L, &nw, &ne, &err)) return 0;
+  return make_plan(*cfg, nw, ne, L).total;
+}
+
+hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspace_bytes,
+                        const uint8_t* host_mask, hyat_handle* out) {
+  if (!out) return HYAT_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg) return HYAT_ERR_INVALID_ARG;
+  const std::string verr = validate_config(*cfg);
+  if (!verr.empty()) return HYAT_ERR_INVALID_ARG;
+  if (cfg->mode == HYAT_MODE_BLOCKMASK && !host_mask) return HYAT_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return HYAT_ERR_INVALID_ARG;
+
+  hyat_ctx* h = new (std::nothrow) hyat_ctx();
+  if (!h) return HYAT_ERR_CUDA;
+  h->cfg = *cfg;
+  h->BH = cfg->B * cfg->H;
+  h->E = cfg->d * cfg->d + cfg->d;
+  h->rq = rows_q(*cfg);
+  h->rk = rows_k(*cfg);
+  int64_t nw = 0, ne = 0;
+  std::string err;
+  if (!plan_counts(*cfg, host_mask, &h->lay, &nw, &ne, &err)) {
+    delete h;
+    return HYAT_ERR_INVALID_ARG;
+  }
+  h->plan = make_plan(*cfg, nw, ne, h->lay);
+  const size_t bound = hyat_workspace_bytes(cfg);
+  if (workspace_bytes < h->plan.total || workspace_bytes < bound) {
+    delete h;
+    return HYAT_ERR_INVALID_ARG;
+  }
+  char* ws = static_cast<char*>(workspace);
+  h->ws = ws;
+  h->d_status = reinterpret_cast<uint32_t*>(ws + h->plan.status);
+  h->d_work = reinterpret_cast<WorkItem*>(ws + h->plan.work);
+  h->d_entries = reinterpret_cast<Entry*>(ws + h->plan.entries);
+  h->d_srest = reinterpret_cast<float*>(ws + h->plan.srest);
+  h->d_srest_t = reinterpret_cast<uint16_t*>(ws + h->plan.srest_t);
+  if (cfg->mode == HYAT_MODE_STREAM) {
+    h->d_ring_k = ws + h->plan.ring_k;
+    h->d_ring_v = ws + h->plan.ring_v;
+    h->d_mask = reinterpret_cast<uint8_t*>(ws + h->plan.mask);
+  } else {
+    h->d_cm = reinterpret_cast<float*>(ws + h->plan.cm);
+    h->d_sseg = reinterpret_cast<float*>(ws + h->plan.sseg);
+  }
+
+  int dev = 0, major = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) {
+    delete h;
+    return HYAT_ERR_CUDA;
+  }
+  h->use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
+              attn_tc_supported(cfg->d, cfg->dtype);
+
+  // layout tables and zeroed state
+  e = cudaMemset(ws, 0, h->plan.status + 256);
+  if (e == cudaSuccess && !h->lay.work.empty())
+    e = cudaMemcpy(h->d_work, h->lay.work.data(), sizeof(WorkItem) * h->lay.work.size(), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && !h->lay.entries.empty())
+    e = cudaMemcpy(h->d_entries, h->lay.entries.data(), sizeof(Entry) * h->lay.entries.size(),
+                   cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && !h->lay.cm.empty())
+    e = cudaMemcpy(h->d_cm, h->lay.cm.data(), sizeof(float) * h->lay.cm.size(), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && cfg->mode == HYAT_MODE_STREAM)
+    e = cudaMemset(ws + h->plan.srest, 0, h->plan.total - h->plan.srest);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    delete h;
+    return HYAT_ERR_CUDA;
+  }
+  *out = h;
+  return HYAT_OK;
+}
+
+hyat_status hyat_destroy(hyat_handle h) {
+  if (!h) return HYAT_OK;
+  for (auto& r : h->recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : h->free_events) cudaEventDestroy(e);
+  delete h;
+  return HYAT_OK;
+}
+
+hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const void* v, void* o,
+                           void* stream) {
+  if (!h) return HYAT_ERR_INVALID_ARG;
+  if (h->cfg.mode == HYAT_MODE_STREAM) return fail(h, HYAT_ERR_INVALID_ARG, "handle is in STREAM mode");
+  hyat_status st = check_ptrs(h, q, k, v, o);
+  if (st != HYAT_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  const Layout& L = h->lay;
+  SegStateArgs sa{};
+  sa.k = k; sa.v = v; sa.rows_per_bh = h->rk;
+  sa.BH = h->BH; sa.d = h->cfg.d; sa.dtype = h->cfg.dtype;
+  sa.nseg = L.nseg; sa.seg_base = 0; sa.seg_stride = L.seg_stride; sa.seg_len = L.seg_len;
+  sa.out = h->d_sseg; sa.accumulate = 0;
+  cudaError_t e = timed(h, K_STATE, s, [&] { return launch_seg_state(sa, s); });
+  if (e != cudaSuccess) return cuda_fail(h, e, "segment state kernel");
+  ComplementArgs ca{};
+  ca.sseg = h->d_sseg; ca.cm = h->d_cm; ca.srest = h->d_srest;
+  ca.BH = h->BH; ca.H = h->cfg.H; ca.cm_heads = L.cm_heads; ca.nseg = L.nseg; ca.nqg = L.nqg; ca.E = h->E;
+  e = timed(h, K_COMPLEMENT, s, [&] { return launch_complement(ca, s); });
+  if (e != cudaSuccess) return cuda_fail(h, e, "complement kernel");
+  return launch_attention(h, attn_args(h, q, k, v, o, h->plan.n_work, L.nqg), s);
+}
+
+hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, const void* v, void* o,
+                                 const uint8_t* host_step_mask, void* stream) {
+  if (!h) return HYAT_ERR_INVALID_ARG;
+  if (h->cfg.mode != HYAT_MODE_STREAM) return fail(h, HYAT_ERR_INVALID_ARG, "handle is not in STREAM mode");
+  hyat_status st = check_ptrs(h, q, k, v, o);
+  if (st != HYAT_OK) return st;
+  const hyat_config& c = h->cfg;
+  const int32_t Lc = stream_chunk_tokens(c), nwc = stream_window_chunks(c), nqt = tiles(Lc);
+  const int32_t s_ = h->step;
+  const int32_t first_visible = std::max(0, s_ - nwc + 1);
+  const int32_t nwin = s_ - first_visible + 1;
+  const int32_t nkt = nqt * nwin;
+  const size_t mask_bytes = size_t(c.mask_heads) * nqt * nkt;
+  if (host_step_mask) {
+    for (int32_t m = 0; m < c.mask_heads; ++m)
+      for (int32_t i = 0; i < nqt; ++i)
+        if (!host_step_mask[(size_t(m) * nqt + i) * nkt + nqt * (nwin - 1) + i])
+          return fail(h, HYAT_ERR_INVALID_ARG, "step mask: diagonal tile of the newest chunk must be kept");
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  cudaError_t e;
+  if (host_step_mask)
+    e = cudaMemcpyAsync(h->d_mask, host_step_mask, mask_bytes, cudaMemcpyHostToDevice, s);
+  else
+    e = cudaMemsetAsync(h->d_mask, 1, mask_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "step mask upload");
+  const int32_t slot = s_ % nwc;
+  e = timed(h, K_FOLD, s, [&]() -> cudaError_t {
+    if (s_ >= nwc) {  // chunk s - nwc leaves the window: fold it into S, z
+      SegStateArgs sa{};
+      sa.k = h->d_ring_k; sa.v = h->d_ring_v; sa.rows_per_bh = h->rk;
+      sa.BH = h->BH; sa.d = c.d; sa.dtype = c.dtype;
+      sa.nseg = 1; sa.seg_base = slot * Lc; sa.seg_stride = Lc; sa.seg_len = Lc;
+      sa.out = h->d_srest; sa.accumulate = 1;
+      cudaError_t e2 = launch_seg_state(sa, s);
+      if (e2 != cudaSuccess) return e2;
+    }
+    RingCopyArgs ra{};
+    ra.k = k; ra.v = v; ra.ring_k = h->d_ring_k; ra.ring_v = h->d_ring_v;
+    ra.BH = h->BH; ra.L = Lc; ra.d = c.d; ra.nslots = nwc; ra.slot = slot;
+    ra.elem_bytes = static_cast<int32_t>(elem_bytes(c));
+    return launch_ring_copy(ra, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(h, e, "stream fold / ring copy");
+  StreamLayoutArgs la{};
+  la.mask = h->d_mask; la.work = h->d_work; la.entries = h->d_entries;
+  la.BH = h->BH; la.H = c.H; la.mask_heads = c.mask_heads; la.nqt = nqt; la.nkt = nkt;
+  la.cap = nqt * nwc; la.L = Lc; la.nwc = nwc; la.first_visible = first_visible;
+  e = timed(h, K_PREP, s, [&] { return launch_stream_layout(la, s); });
+  if (e != cudaSuccess) return cuda_fail(h, e, "stream layout kernel");
+  st = launch_attention(h, attn_args(h, q, h->d_ring_k, h->d_ring_v, o, int64_t(h->BH) * nqt, 1), s);
+  if (st != HYAT_OK) return st;
+  h->step += 1;
+  return HYAT_OK;
+}
+
+hyat_status hyat_sync(hyat_handle h) {
+  if (!h) return HYAT_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize(h->last_stream);
+  if (e != cudaSuccess) return cuda_fail(h, e, "stream synchronize");
+  uint32_t status = 0;
+  e = cudaMemcpy(&status, h->d_status, sizeof(status), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "status read");
+  if (status) {
+    cudaMemset(h->d_status, 0, sizeof(status));
+    if (status & kStatusTimeout) return fail(h, HYAT_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");
+    return fail(h, HYAT_ERR_DEVICE_TIMEOUT, "a device-side bounds check failed");
+  }
+  return HYAT_OK;
+}
+
+hyat_status hyat_plan_layout(const hyat_config* cfg, const uint8_t* host_mask, int32_t* work, size_t work_cap,
+                             int32_t* entries, size_t entries_cap, int64_t* counts) {
+  if (!cfg || !counts) return HYAT_ERR_INVALID_ARG;
+  if (!validate_config(*cfg).empty() || cfg->mode == HYAT_MODE_STREAM) return HYAT_ERR_INVALID_ARG;
+  if (cfg->mode == HYAT_MODE_BLOCKMASK && !host_mask) return HYAT_ERR_INVALID_ARG;
+  Layout L;
+  if (!build_layout(*cfg, host_mask, &L).empty()) return HYAT_ERR_INVALID_ARG;
+  counts[0] = static_cast<int64_t>(L.work.size());
+  counts[1] = static_cast<int64_t>(L.entries.size());
+  if (!work || !entries) return HYAT_OK;  // size query
+  if (work_cap < L.work.size() * 8 || entries_cap < L.entries.size() * 2) return HYAT_ERR_INVALID_ARG;
+  std::memcpy(work, L.work.data(), sizeof(WorkItem) * L.work.size());
+  std::memcpy(entries, L.entries.data(), sizeof(Entry) * L.entries.size());
+  return HYAT_OK;
+}
+
+hyat_status hyat_radial_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t* out, size_t out_bytes) {
+  if (n_frames < 1 || tokens_per_frame < 1 || !out) return HYAT_ERR_INVALID_ARG;
+  const int64_t nT = tiles(int64_t(n_frames) * tokens_per_frame);
+  if (out_bytes < size_t(nT * nT)) return HYAT_ERR_INVALID_ARG;
+  radial_tile_mask(n_frames, tokens_per_frame, out);
+  return HYAT_OK;
+}
+
+hyat_status hyat_stream_plan(const hyat_config* cfg, int32_t step, int32_t* info, size_t info_len) {
+  if (!cfg || !info || step < 0 || cfg->mode != HYAT_MODE_STREAM || !validate_config(*cfg).empty())
+    return HYAT_ERR_INVALID_ARG;
+  const int32_t nwc = stream_window_chunks(*cfg);
+  if (info_len < size_t(4 + nwc)) return HYAT_ERR_INVALID_ARG;
+  const int32_t first = std::max(0, step - nwc + 1);
+  info[0] = first;
+  info[1] = step - first + 1;
+  info[2] = step >= nwc ? step - nwc : -1;
+  info[3] = step % nwc;
+  for (int32_t w = 0; w < nwc; ++w) info[4 + w] = w < info[1] ? (first + w) % nwc : -1;
+  return HYAT_OK;
+}
+
+// state blob: header, then S/z (fp32 [BH][E]), ring K, ring V
+namespace {
+struct StateHeader {
+  uint32_t magic, version;
+  int32_t step, BH, d, L, nwc, dtype;
+};
+constexpr uint32_t kMagic = 0x54415948u;  // "HYAT"
+}  // namespace
+
+size_t hyat_stream_state_bytes(hyat_handle h) {
+  if (!h || h->cfg.mode != HYAT_MODE_STREAM) return 0;
+  const size_t ring = size_t(h->BH) * stream_window_chunks(h->cfg) * stream_chunk_tokens(h->cfg) * h->cfg.d *
+                      elem_bytes(h->cfg);
+  return sizeof(StateHeader) + sizeof(float) * size_t(h->BH) * h->E + 2 * ring;
+}
+
+hyat_status hyat_stream_get_state(hyat_handle h, void* dst_host, size_t bytes) {
+  if (!h || !dst_host) return HYAT_ERR_INVALID_ARG;
+  if (h->cfg.mode != HYAT_MODE_STREAM) return fail(h, HYAT_ERR_INVALID_ARG, "handle is not in STREAM mode");
+  if (bytes < hyat_stream_state_bytes(h)) return fail(h, HYAT_ERR_INVALID_ARG, "state buffer too small");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(h, e, "synchronize");
+  StateHeader hd{kMagic, 1, h->step, h->BH, h->cfg.d, stream_chunk_tokens(h->cfg), stream_window_chunks(h->cfg),
+                 h->cfg.dtype};
+  char* p = static_cast<char*>(dst_host);
+  std::memcpy(p, &hd, sizeof(hd));
+  p += sizeof(hd);
+  const size_t sb = sizeof(float) * size_t(h->BH) * h->E;
+  const size_t rb = (hyat_stream_state_bytes(h) - sizeof(hd) - sb) / 2;
+  e = cudaMemcpy(p, h->d_srest, sb, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(p + sb, h->d_ring_k, rb, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(p + sb + rb, h->d_ring_v, rb, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "state copy");
+  return HYAT_OK;
+}
+
+hyat_status hyat_stream_set_state(hyat_handle h, const void* src_host, size_t bytes) {
+  if (!h || !src_host) return HYAT_ERR_INVALID_ARG;
+  if (h->cfg.mode != HYAT_MODE_STREAM) return fail(h, HYAT_ERR_INVALID_ARG, "handle is not in STREAM mode");
+  if (bytes < hyat_stream_state_bytes(h)) return fail(h, HYAT_ERR_STATE, "state buffer too small");
+  StateHeader hd;
+  std::memcpy(&hd, src_host, sizeof(hd));
+  if (hd.magic != kMagic || hd.version != 1 || hd.BH != h->BH || hd.d != h->cfg.d ||
+      hd.L != stream_chunk_tokens(h->cfg) || hd.nwc != stream_window_chunks(h->cfg) || hd.dtype != h->cfg.dtype ||
+      hd.step < 0)
+    return fail(h, HYAT_ERR_STATE, "state blob does not match this handle");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(h, e, "synchronize");
+  const char* p = static_cast<const char*>(src_host) + sizeof(hd);
+  const size_t sb = sizeof(float) * size_t(h->BH) * h->E;
+  const size_t rb = (hyat_stream_state_bytes(h) - sizeof(hd) - sb) / 2;
+  e = cudaMemcpy(h->d_srest, p, sb, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->d_ring_k, p + sb, rb, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(h->d_ring_v, p + sb + rb, rb, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(h, e, "state copy");
+  h->step = hd.step;
+  return HYAT_OK;
+}
+
+hyat_status hyat_set_profiling(hyat_handle h, int enable) {
+  if (!h) return HYAT_ERR_INVALID_ARG;
+  h->profiling = enable != 0;
+  return HYAT_OK;
+}
+
+hyat_status hyat_kernel_times(hyat_handle h, double* ms, int64_t* launches, int n_kinds) {
+  if (!h || !ms || !launches || n_kinds < 1) return HYAT_ERR_INVALID_ARG;
+  for (auto& r : h->recs) {
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(h, e, "event synchronize");
+    float t = 0.0f;
+    e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(h, e, "event elapsed time");
+    h->ms[r.kind] += t;
+    h->launches[r.kind] += 1;
+    h->free_events.push_back(r.a);
+    h->free_events.push_back(r.b);
+  }
+  h->recs.clear();
+  for (int i = 0; i < n_kinds; ++i) {
+    ms[i] = i < kKinds ? h->ms[i] : 0.0;
+    launches[i] = i < kKinds ? h->launches[i] : 0;
+  }
+  for (int i = 0; i < kKinds; ++i) {
+    h->ms[i] = 0.0;
+    h->launches[i] = 0;
+  }
+  return HYAT_OK;
+}
+
+}  // extern "C"

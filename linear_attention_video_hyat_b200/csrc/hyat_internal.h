@@ -1,0 +1,108 @@
+// Internal declarations shared by the host runtime and the kernels of libhyat.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/hyat.h"
+
+namespace hyat {
+
+constexpr int kTile = 128;          // query / key tile edge (rows)
+
+// Device status word bits (workspace offset 0).
+constexpr uint32_t kStatusTimeout = 1u;     // a bounded wait gave up
+constexpr uint32_t kStatusBadTile = 2u;     // a tile descriptor failed its bounds check
+
+// A work item: one query tile and the key tiles of its softmax window.
+struct WorkItem {
+  int32_t bh, q_row, q_len, state_group, entry_begin, entry_end, pad0, pad1;
+};
+static_assert(sizeof(WorkItem) == 32, "work item is 8 int32");
+
+// A key tile of a window: rows [k_row, k_row + k_len) of one (b, h).
+struct Entry {
+  int32_t k_row, k_len;
+};
+
+// Host-side layout of a configuration.
+struct Layout {
+  // uniform key segments whose linear states are formed: segment g covers
+  // rows [seg_base + g * seg_stride, + min(seg_len, rows_k - start))
+  int32_t nseg = 0, seg_stride = 0, seg_len = 0;
+  int32_t nqg = 0;                 // state groups (chunks, query tiles or 1)
+  int32_t cm_heads = 1;            // heads of the complement matrix
+  std::vector<float> cm;           // [cm_heads][nqg][nseg]: 1 = segment is in the linear set
+  std::vector<WorkItem> work;
+  std::vector<Entry> entries;
+};
+
+// Validate a configuration; returns an empty string if valid.
+std::string validate_config(const hyat_config& c);
+int64_t rows_q(const hyat_config& c);           // query rows per (b, h)
+int64_t rows_k(const hyat_config& c);           // key rows per (b, h) (ring for STREAM)
+int32_t stream_chunk_tokens(const hyat_config& c);
+int32_t stream_window_chunks(const hyat_config& c);
+int32_t tiles(int64_t rows);
+
+// Host layout builders (layout.cpp).
+std::string build_layout(const hyat_config& c, const uint8_t* host_mask, Layout* out);
+void radial_tile_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t* out);
+
+// ---- kernel launch wrappers (kernels_simt.cu, attn_tc.cu) ----
+struct SegStateArgs {
+  const void* k; const void* v; int64_t rows_per_bh;
+  int32_t BH, d, dtype;
+  int32_t nseg, seg_base, seg_stride, seg_len;
+  float* out;                 // [BH][nseg][E], E = d*d + d (S row-major [a][b], then z[a])
+  int32_t accumulate;         // out += instead of out =
+};
+cudaError_t launch_seg_state(const SegStateArgs& a, cudaStream_t s);
+
+struct ComplementArgs {
+  const float* sseg;          // [BH][nseg][E]
+  const float* cm;            // [cm_heads][nqg][nseg]
+  float* srest;               // [BH][nqg][E]
+  int32_t BH, H, cm_heads, nseg, nqg, E;
+};
+cudaError_t launch_complement(const ComplementArgs& a, cudaStream_t s);
+
+// S (fp32 [a][b] then z) -> bf16 S^T [b][a] for the tensor-core linear term.
+cudaError_t launch_state_transpose_bf16(const float* srest, uint16_t* st, int64_t n_groups,
+                                        int32_t d, cudaStream_t s);
+
+struct AttnArgs {
+  const void* q; const void* k; const void* v; void* o;
+  int64_t q_rows, k_rows;     // rows per (b, h)
+  const WorkItem* work; int32_t n_work;
+  const Entry* entries;
+  const float* srest;         // [BH][nqg][E]
+  const uint16_t* srest_t;    // [BH][nqg][d][d] bf16 (tensor-core path)
+  int32_t nqg, d, dtype, BH;
+  float scale_log2;           // scale * log2(e)
+  uint32_t* status;
+};
+cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s);
+bool attn_tc_supported(int d, int dtype);
+
+struct RingCopyArgs {
+  const void* k; const void* v;   // [BH][L][d]
+  void* ring_k; void* ring_v;     // [BH][nslots][L][d]
+  int32_t BH, L, d, nslots, slot, elem_bytes;
+};
+cudaError_t launch_ring_copy(const RingCopyArgs& a, cudaStream_t s);
+
+struct StreamLayoutArgs {
+  const uint8_t* mask;            // [mask_heads][nqt][nkt] (device)
+  WorkItem* work;                 // [BH][nqt]
+  Entry* entries;                 // [BH][nqt][cap]
+  int32_t BH, H, mask_heads, nqt, nkt, cap, L, nwc, first_visible;
+};
+cudaError_t launch_stream_layout(const StreamLayoutArgs& a, cudaStream_t s);
+
+}  // namespace hyat

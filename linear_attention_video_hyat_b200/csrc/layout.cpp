@@ -1,0 +1,201 @@
+// Host layout builder: which key tiles each query tile attends to by softmax,
+// and which key segments reach it through the linear state.
+//
+// Window rules follow the hybrid attention of ReHyAt (Abstract: chunk-wise
+// softmax + linear attention) and the block-sparse window of Hybrid Forcing
+// (Section 2.A); the radial mask follows Radial Attention (Abstract: each
+// token attends to spatially near tokens, the window shrinking with temporal
+// distance).
+#include <algorithm>
+#include <cmath>
+#include <string>
+
+#include "hyat_internal.h"
+
+namespace hyat {
+
+int32_t tiles(int64_t rows) { return static_cast<int32_t>((rows + kTile - 1) / kTile); }
+
+int32_t stream_chunk_tokens(const hyat_config& c) { return c.chunk_frames * c.tokens_per_frame; }
+int32_t stream_window_chunks(const hyat_config& c) { return c.window_frames / c.chunk_frames; }
+
+int64_t rows_q(const hyat_config& c) {
+  if (c.mode == HYAT_MODE_STREAM) return stream_chunk_tokens(c);
+  return static_cast<int64_t>(c.n_frames) * c.tokens_per_frame;
+}
+
+int64_t rows_k(const hyat_config& c) {
+  if (c.mode == HYAT_MODE_STREAM)
+    return static_cast<int64_t>(stream_window_chunks(c)) * stream_chunk_tokens(c);
+  return static_cast<int64_t>(c.n_frames) * c.tokens_per_frame;
+}
+
+std::string validate_config(const hyat_config& c) {
+  if (c.B < 1 || c.H < 1) return "B and H must be >= 1";
+  if (c.d != 64 && c.d != 128) return "d must be 64 or 128";
+  if (c.tokens_per_frame < 1) return "tokens_per_frame must be >= 1";
+  if (c.dtype != HYAT_F32 && c.dtype != HYAT_BF16) return "dtype must be HYAT_F32 or HYAT_BF16";
+  if (c.phi != HYAT_PHI_ELU1) return "phi must be HYAT_PHI_ELU1";
+  if (!(c.scale >= 0.0f) || std::isinf(c.scale)) return "scale must be finite and >= 0";
+  switch (c.mode) {
+    case HYAT_MODE_WINDOW:
+      if (c.n_frames < 1) return "n_frames must be >= 1";
+      if (c.chunk_frames < 1) return "chunk_frames must be >= 1";
+      if (c.halo_frames < 0) return "halo_frames must be >= 0";
+      break;
+    case HYAT_MODE_BLOCKMASK:
+      if (c.n_frames < 1) return "n_frames must be >= 1";
+      if (c.mask_heads != 1 && c.mask_heads != c.H) return "mask_heads must be 1 or H";
+      break;
+    case HYAT_MODE_RADIAL:
+      if (c.n_frames < 1) return "n_frames must be >= 1";
+      break;
+    case HYAT_MODE_STREAM:
+      if (c.chunk_frames < 1) return "chunk_frames must be >= 1";
+      if (c.window_frames < c.chunk_frames || c.window_frames % c.chunk_frames != 0)
+        return "window_frames must be a positive multiple of chunk_frames";
+      if (c.mask_heads != 1 && c.mask_heads != c.H) return "mask_heads must be 1 or H";
+      break;
+    default:
+      return "unknown mode";
+  }
+  const int64_t n = rows_k(c) > rows_q(c) ? rows_k(c) : rows_q(c);
+  if (n * c.d >= (int64_t(1) << 31)) return "rows * d per head must be < 2^31";
+  if (static_cast<int64_t>(c.B) * c.H * n * c.d >= (int64_t(1) << 40)) return "tensor too large";
+  return "";
+}
+
+// Radial tile mask by interval marking: for every query tile and every
+// frame piece it covers, the keys near that piece in key frame fk form one
+// position interval [p0 - r, p1 + r] (r = largest integer with 2r < w); the
+// tiles that interval touches are kept.
+void radial_tile_mask(int32_t n_frames, int32_t F, uint8_t* out) {
+  const int64_t N = static_cast<int64_t>(n_frames) * F;
+  const int32_t nT = tiles(N);
+  std::fill(out, out + static_cast<size_t>(nT) * nT, uint8_t(0));
+  for (int32_t a = 0; a < nT; ++a) {
+    const int64_t r0 = static_cast<int64_t>(a) * kTile;
+    const int64_t r1 = std::min<int64_t>(N, r0 + kTile);  // exclusive
+    for (int64_t r = r0; r < r1;) {
+      const int32_t fq = static_cast<int32_t>(r / F);
+      const int64_t piece_end = std::min<int64_t>(r1, static_cast<int64_t>(fq + 1) * F);
+      const int64_t p0 = r - static_cast<int64_t>(fq) * F;
+      const int64_t p1 = piece_end - 1 - static_cast<int64_t>(fq) * F;
+      for (int32_t fk = 0; fk < n_frames; ++fk) {
+        const int32_t t = fq > fk ? fq - fk : fk - fq;
+        int64_t lo, hi;  // key positions inside frame fk, inclusive
+        if (t == 0) {
+          lo = 0;
+          hi = F - 1;
+        } else {
+          int lg = 0;
+          while ((2 << lg) <= t) ++lg;           // floor(log2 t)
+          const int64_t w = static_cast<int64_t>(F) >> lg;
+          if (w <= 0) continue;
+          const int64_t rad = (w - 1) / 2;        // 2*|dp| < w  <=>  |dp| <= (w-1)/2
+          lo = std::max<int64_t>(0, p0 - rad);
+          hi = std::min<int64_t>(F - 1, p1 + rad);
+          if (lo > hi) continue;
+        }
+        const int64_t k0 = static_cast<int64_t>(fk) * F + lo;
+        const int64_t k1 = static_cast<int64_t>(fk) * F + hi;
+        for (int64_t b = k0 / kTile; b <= k1 / kTile; ++b) out[static_cast<size_t>(a) * nT + b] = 1;
+      }
+      r = piece_end;
+    }
+  }
+}
+
+static void push_window_entries(int64_t k_lo, int64_t k_hi, std::vector<Entry>* e) {
+  for (int64_t k = k_lo; k < k_hi; k += kTile)
+    e->push_back(Entry{static_cast<int32_t>(k), static_cast<int32_t>(std::min<int64_t>(kTile, k_hi - k))});
+}
+
+std::string build_layout(const hyat_config& c, const uint8_t* host_mask, Layout* L) {
+  *L = Layout();
+  const int32_t BH = c.B * c.H;
+  const int64_t N = rows_q(c);
+  const int32_t F = c.tokens_per_frame;
+  if (c.mode == HYAT_MODE_WINDOW) {
+    const int32_t T = c.n_frames, C = c.chunk_frames, h = c.halo_frames;
+    const int32_t n_chunks = (T + C - 1) / C;
+    L->nseg = T;
+    L->seg_stride = F;
+    L->seg_len = F;
+    L->nqg = n_chunks;
+    L->cm_heads = 1;
+    L->cm.assign(static_cast<size_t>(n_chunks) * T, 0.0f);
+    std::vector<int32_t> eb(n_chunks), ee(n_chunks);
+    for (int32_t ch = 0; ch < n_chunks; ++ch) {
+      const int32_t lo = std::max(0, ch * C - h);
+      const int32_t hi = std::min(T, (ch + 1) * C + h);
+      for (int32_t f = 0; f < T; ++f)
+        L->cm[static_cast<size_t>(ch) * T + f] = (f < lo || f >= hi) ? 1.0f : 0.0f;
+      eb[ch] = static_cast<int32_t>(L->entries.size());
+      push_window_entries(static_cast<int64_t>(lo) * F, static_cast<int64_t>(hi) * F, &L->entries);
+      ee[ch] = static_cast<int32_t>(L->entries.size());
+    }
+    for (int32_t bh = 0; bh < BH; ++bh)
+      for (int32_t ch = 0; ch < n_chunks; ++ch) {
+        const int64_t q0 = static_cast<int64_t>(ch) * C * F;
+        const int64_t q1 = std::min<int64_t>(N, static_cast<int64_t>(ch + 1) * C * F);
+        for (int64_t q = q0; q < q1; q += kTile)
+          L->work.push_back(WorkItem{bh, static_cast<int32_t>(q),
+                                     static_cast<int32_t>(std::min<int64_t>(kTile, q1 - q)), ch,
+                                     eb[ch], ee[ch], 0, 0});
+      }
+    return "";
+  }
+  if (c.mode == HYAT_MODE_BLOCKMASK || c.mode == HYAT_MODE_RADIAL) {
+    const int32_t nT = tiles(N);
+    std::vector<uint8_t> radial;
+    const uint8_t* mask = host_mask;
+    int32_t mh = c.mask_heads;
+    if (c.mode == HYAT_MODE_RADIAL) {
+      radial.resize(static_cast<size_t>(nT) * nT);
+      radial_tile_mask(c.n_frames, F, radial.data());
+      mask = radial.data();
+      mh = 1;
+    } else if (mask == nullptr) {
+      return "BLOCKMASK needs a host mask";
+    }
+    L->nseg = nT;
+    L->seg_stride = kTile;
+    L->seg_len = kTile;
+    L->nqg = nT;
+    L->cm_heads = mh;
+    L->cm.assign(static_cast<size_t>(mh) * nT * nT, 0.0f);
+    std::vector<int32_t> eb(static_cast<size_t>(mh) * nT), ee(static_cast<size_t>(mh) * nT);
+    for (int32_t m = 0; m < mh; ++m)
+      for (int32_t i = 0; i < nT; ++i) {
+        const size_t row = (static_cast<size_t>(m) * nT + i) * nT;
+        eb[static_cast<size_t>(m) * nT + i] = static_cast<int32_t>(L->entries.size());
+        for (int32_t b = 0; b < nT; ++b) {
+          if (mask[row + b]) {
+            L->entries.push_back(Entry{b * kTile, static_cast<int32_t>(std::min<int64_t>(kTile, N - int64_t(b) * kTile))});
+          } else {
+            L->cm[row + b] = 1.0f;
+          }
+        }
+        ee[static_cast<size_t>(m) * nT + i] = static_cast<int32_t>(L->entries.size());
+      }
+    for (int32_t bh = 0; bh < BH; ++bh) {
+      const int32_t m = (mh == 1) ? 0 : bh % c.H;
+      for (int32_t i = 0; i < nT; ++i)
+        L->work.push_back(WorkItem{bh, i * kTile, static_cast<int32_t>(std::min<int64_t>(kTile, N - int64_t(i) * kTile)),
+                                   i, eb[static_cast<size_t>(m) * nT + i], ee[static_cast<size_t>(m) * nT + i], 0, 0});
+    }
+    return "";
+  }
+  if (c.mode == HYAT_MODE_STREAM) {
+    // work items and entries are produced on the device each step
+    L->nseg = 1;
+    L->seg_stride = stream_chunk_tokens(c);
+    L->seg_len = stream_chunk_tokens(c);
+    L->nqg = 1;
+    return "";
+  }
+  return "unknown mode";
+}
+
+}  // namespace hyat

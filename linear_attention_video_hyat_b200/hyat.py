@@ -1,0 +1,233 @@
+"""Thin ctypes binding of libhyat (include/hyat.h).
+
+Only argument marshalling lives here: every step of the forward pass runs in
+the library's CUDA kernels. PyTorch supplies device memory (tensors and the
+workspace) and the current CUDA stream. If the compiled library is missing the
+import fails loudly; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhyat.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_STATE = range(6)
+F32, BF16 = 0, 1
+MODE_WINDOW, MODE_BLOCKMASK, MODE_RADIAL, MODE_STREAM = range(4)
+FLAG_SIMT = 1
+TILE = 128
+KERNEL_KINDS = ("state", "complement", "attention", "fold_ring", "layout_prep")
+
+_MODES = {"window": MODE_WINDOW, "blockmask": MODE_BLOCKMASK, "radial": MODE_RADIAL, "stream": MODE_STREAM}
+
+EXPORTED = (
+    "hyat_workspace_bytes", "hyat_create", "hyat_fwd_bidir", "hyat_fwd_stream_step", "hyat_sync",
+    "hyat_destroy", "hyat_last_error", "hyat_status_string", "hyat_plan_layout", "hyat_radial_mask",
+    "hyat_stream_plan", "hyat_stream_state_bytes", "hyat_stream_get_state", "hyat_stream_set_state",
+    "hyat_set_profiling", "hyat_kernel_times",
+)
+
+
+class HyatError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"hyat status {status}: {msg}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("tokens_per_frame", ctypes.c_int32), ("n_frames", ctypes.c_int32),
+        ("chunk_frames", ctypes.c_int32), ("halo_frames", ctypes.c_int32),
+        ("window_frames", ctypes.c_int32), ("mode", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("phi", ctypes.c_int32), ("mask_heads", ctypes.c_int32), ("flags", ctypes.c_uint32),
+        ("scale", ctypes.c_float),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libhyat.so not built ({LIB_PATH}); run "
+                          f"`python -m linear_attention_video_hyat_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, S, I32, I64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64
+    CP = ctypes.POINTER(Config)
+    sig = {
+        "hyat_workspace_bytes": (S, [CP]),
+        "hyat_create": (ctypes.c_int, [CP, P, S, P, ctypes.POINTER(P)]),
+        "hyat_fwd_bidir": (ctypes.c_int, [P, P, P, P, P, P]),
+        "hyat_fwd_stream_step": (ctypes.c_int, [P, P, P, P, P, P, P]),
+        "hyat_sync": (ctypes.c_int, [P]),
+        "hyat_destroy": (ctypes.c_int, [P]),
+        "hyat_last_error": (ctypes.c_char_p, [P]),
+        "hyat_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "hyat_plan_layout": (ctypes.c_int, [CP, P, P, S, P, S, ctypes.POINTER(I64)]),
+        "hyat_radial_mask": (ctypes.c_int, [I32, I32, P, S]),
+        "hyat_stream_plan": (ctypes.c_int, [CP, I32, P, S]),
+        "hyat_stream_state_bytes": (S, [P]),
+        "hyat_stream_get_state": (ctypes.c_int, [P, P, S]),
+        "hyat_stream_set_state": (ctypes.c_int, [P, P, S]),
+        "hyat_set_profiling": (ctypes.c_int, [P, ctypes.c_int]),
+        "hyat_kernel_times": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64), ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def make_config(mode, B, H, d, tokens_per_frame, n_frames=0, chunk_frames=1, halo_frames=0,
+                window_frames=0, dtype=BF16, mask_heads=1, flags=0, scale=0.0) -> Config:
+    m = _MODES[mode] if isinstance(mode, str) else int(mode)
+    dt = {"f32": F32, "bf16": BF16}.get(dtype, dtype) if isinstance(dtype, str) else int(dtype)
+    return Config(B, H, d, tokens_per_frame, n_frames, chunk_frames, halo_frames, window_frames,
+                  m, dt, 0, mask_heads, flags, float(scale))
+
+
+def config_from_workload(w, flags=0, mask_heads=1) -> Config:
+    return make_config(w.mode, w.B, w.H, w.d, w.tokens_per_frame, w.n_frames, w.chunk_frames,
+                       w.halo_frames, w.window_frames, w.dtype, mask_heads=mask_heads, flags=flags)
+
+
+def _check(status, handle=None):
+    if status != OK:
+        msg = lib.hyat_last_error(handle).decode() if handle else lib.hyat_status_string(status).decode()
+        raise HyatError(status, msg)
+
+
+def _u8(arr) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(arr), dtype=np.uint8)
+
+
+# ---------------------------------------------------------------- host hooks
+def workspace_bytes(cfg: Config) -> int:
+    return int(lib.hyat_workspace_bytes(ctypes.byref(cfg)))
+
+
+def plan_layout(cfg: Config, mask=None):
+    """Host-only layout: (work [n,8] int32, entries [m,2] int32)."""
+    counts = (ctypes.c_int64 * 2)()
+    m = None if mask is None else _u8(mask)
+    mp = None if m is None else m.ctypes.data
+    _check(lib.hyat_plan_layout(ctypes.byref(cfg), mp, None, 0, None, 0, counts))
+    work = np.zeros((counts[0], 8), np.int32)
+    ent = np.zeros((max(counts[1], 1), 2), np.int32)
+    _check(lib.hyat_plan_layout(ctypes.byref(cfg), mp, work.ctypes.data, work.size,
+                                ent.ctypes.data, ent.size, counts))
+    return work, ent[:counts[1]]
+
+
+def radial_mask(n_frames: int, tokens_per_frame: int) -> np.ndarray:
+    nT = -(-n_frames * tokens_per_frame // TILE)
+    out = np.zeros((nT, nT), np.uint8)
+    _check(lib.hyat_radial_mask(n_frames, tokens_per_frame, out.ctypes.data, out.size))
+    return out
+
+
+def stream_plan(cfg: Config, step: int):
+    nwc = cfg.window_frames // cfg.chunk_frames
+    info = np.zeros(4 + nwc, np.int32)
+    _check(lib.hyat_stream_plan(ctypes.byref(cfg), step, info.ctypes.data, info.size))
+    return {"first_visible": int(info[0]), "n_visible": int(info[1]), "evicted": int(info[2]),
+            "write_slot": int(info[3]), "slots": [int(x) for x in info[4:4 + info[1]]]}
+
+
+# ---------------------------------------------------------------- device API
+class Hyat:
+    """A handle bound to one configuration, its workspace and (for STREAM) its state."""
+
+    def __init__(self, cfg: Config, mask=None, device=None):
+        if not torch.cuda.is_available():
+            raise RuntimeError("libhyat needs a CUDA device")
+        self.cfg = cfg
+        self.device = torch.device(device if device is not None else "cuda")
+        nbytes = workspace_bytes(cfg)
+        if nbytes == 0:
+            raise HyatError(ERR_INVALID_ARG, "invalid configuration")
+        with torch.cuda.device(self.device):
+            self.workspace = torch.empty(nbytes + 256, dtype=torch.uint8, device=self.device)
+            off = (-self.workspace.data_ptr()) % 256
+            self._ws_ptr = self.workspace.data_ptr() + off
+            self._mask = None if mask is None else _u8(mask)
+            h = ctypes.c_void_p()
+            st = lib.hyat_create(ctypes.byref(cfg), self._ws_ptr, nbytes,
+                                 None if self._mask is None else self._mask.ctypes.data, ctypes.byref(h))
+            _check(st)
+        self.handle = h
+        self.dtype = torch.float32 if cfg.dtype == F32 else torch.bfloat16
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib.hyat_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check_t(self, t, name, rows):
+        c = self.cfg
+        if t.device.type != "cuda" or t.dtype != self.dtype or not t.is_contiguous():
+            raise ValueError(f"{name}: need a contiguous {self.dtype} CUDA tensor")
+        if tuple(t.shape) != (c.B, c.H, rows, c.d):
+            raise ValueError(f"{name}: shape {tuple(t.shape)} != {(c.B, c.H, rows, c.d)}")
+
+    def forward(self, q, k, v, out=None, stream=None):
+        c = self.cfg
+        n = c.tokens_per_frame * c.n_frames
+        for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_t(t, nm, n)
+        out = torch.empty_like(q) if out is None else out
+        self._check_t(out, "out", n)
+        s = torch.cuda.current_stream(q.device) if stream is None else stream
+        _check(lib.hyat_fwd_bidir(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  s.cuda_stream), self.handle)
+        return out
+
+    def stream_step(self, q, k, v, mask=None, out=None, stream=None):
+        c = self.cfg
+        L = c.chunk_frames * c.tokens_per_frame
+        for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_t(t, nm, L)
+        out = torch.empty_like(q) if out is None else out
+        self._check_t(out, "out", L)
+        m = None if mask is None else _u8(mask)
+        s = torch.cuda.current_stream(q.device) if stream is None else stream
+        _check(lib.hyat_fwd_stream_step(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        None if m is None else m.ctypes.data, s.cuda_stream), self.handle)
+        return out
+
+    def sync(self):
+        _check(lib.hyat_sync(self.handle), self.handle)
+
+    def get_state(self) -> bytes:
+        n = lib.hyat_stream_state_bytes(self.handle)
+        buf = ctypes.create_string_buffer(n)
+        _check(lib.hyat_stream_get_state(self.handle, ctypes.addressof(buf), n), self.handle)
+        return buf.raw
+
+    def set_state(self, blob: bytes):
+        buf = ctypes.create_string_buffer(blob, len(blob))
+        _check(lib.hyat_stream_set_state(self.handle, ctypes.addressof(buf), len(blob)), self.handle)
+
+    def set_profiling(self, on: bool):
+        _check(lib.hyat_set_profiling(self.handle, 1 if on else 0), self.handle)
+
+    def kernel_times(self):
+        n = len(KERNEL_KINDS)
+        ms = (ctypes.c_double * n)()
+        cnt = (ctypes.c_int64 * n)()
+        _check(lib.hyat_kernel_times(self.handle, ms, cnt, n), self.handle)
+        return {k: (ms[i], cnt[i]) for i, k in enumerate(KERNEL_KINDS)}

@@ -1,0 +1,241 @@
+"""GPU parity of libhyat against the fp64 oracle, through the C ABI.
+
+Small geometries compare every output element; they span several 128-row
+tiles with ragged tails (frames and chunks that are not multiples of 128).
+The full-size workloads compare sampled rows (first and last rows of query
+tiles, chunk edges, random rows) that the oracle evaluates one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_video_hyat_b200 import hyat, workloads as wl
+from parity import assert_parity, f64, sample_rows, errors
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(*ts):
+    return [t.cuda() for t in ts]
+
+
+def _bidir(w, mask=None, flags=0, mask_heads=1, qkv=None):
+    cfg = hyat.config_from_workload(w, flags=flags, mask_heads=mask_heads)
+    q, k, v = wl.gen_qkv(w) if qkv is None else qkv
+    h = hyat.Hyat(cfg, mask)
+    o = h.forward(*_dev(q, k, v))
+    h.sync()
+    out = o.cpu()
+    h.close()
+    return out, (q, k, v)
+
+
+def _window_ref(w, q, k, v, rows=None):
+    return oracle.bidir_window_attention(f64(q), f64(k), f64(v), w.tokens_per_frame, w.n_frames,
+                                         w.chunk_frames, w.halo_frames, rows=rows)
+
+
+# ------------------------------------------------------------------ small, full output
+def test_tiny_f32_workload_full():
+    w = wl.TINY_F32
+    o, (q, k, v) = _bidir(w)
+    assert_parity("f32", f64(o), _window_ref(w, q, k, v), w.name)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("T,F,C,h,d,H", [(7, 200, 2, 1, 128, 2), (5, 300, 3, 1, 64, 3), (4, 64, 1, 0, 128, 2),
+                                         (3, 130, 3, 0, 128, 1), (6, 1560, 3, 1, 128, 1)])
+def test_window_small(dtype, T, F, C, h, d, H):
+    w = wl.Workload("small", "window", 1, H, d, F, T, C, h, dtype=dtype, seed=T * 1000 + F)
+    o, (q, k, v) = _bidir(w)
+    assert_parity(dtype, f64(o), _window_ref(w, q, k, v), (T, F, C, h, d, H))
+
+
+def test_window_batch2_per_head_std():
+    w = wl.Workload("small_b2", "window", 2, 3, 128, 250, 6, 3, 1, per_head_std=True, seed=11)
+    o, (q, k, v) = _bidir(w)
+    assert_parity("bf16", f64(o), _window_ref(w, q, k, v), w.name)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("kind", ["random", "zeros", "ones"])
+def test_blockmask_small(dtype, kind):
+    T, F, H = 5, 230, 2
+    N = T * F
+    nT = -(-N // 128)
+    mask = {"random": wl.gen_tile_mask(H, nT, nT, seed=4),
+            "zeros": np.zeros((H, nT, nT), np.uint8),
+            "ones": np.ones((H, nT, nT), np.uint8)}[kind]
+    w = wl.Workload("bm", "blockmask", 1, H, 128, F, T, dtype=dtype, seed=5)
+    o, (q, k, v) = _bidir(w, mask=mask, mask_heads=H)
+    ref = oracle.blockmask_attention(f64(q), f64(k), f64(v), mask)
+    assert_parity(dtype, f64(o), ref, kind)
+    if kind == "ones":      # window = all tokens: exact softmax attention
+        sdpa = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(f64(q)), torch.from_numpy(f64(k)), torch.from_numpy(f64(v))).numpy()
+        assert_parity(dtype, f64(o), sdpa, "ones vs sdpa")
+    if kind == "zeros":     # empty window: pure linear attention
+        pq, pk = oracle.phi_elu1(f64(q)), oracle.phi_elu1(f64(k))
+        S = np.einsum("bhna,bhnc->bhac", pk, f64(v))
+        lin = np.einsum("bhna,bhac->bhnc", pq, S) / np.einsum("bhna,bha->bhn", pq, pk.sum(2))[..., None]
+        assert_parity(dtype, f64(o), lin, "zeros vs linear")
+
+
+@pytest.mark.parametrize("T,F", [(9, 300), (6, 200)])
+def test_radial_small(T, F):
+    w = wl.Workload("radial_small", "radial", 1, 2, 128, F, T, seed=6)
+    o, (q, k, v) = _bidir(w)
+    ref = oracle.radial_attention(f64(q), f64(k), f64(v), T, F)
+    assert_parity("bf16", f64(o), ref, w.name)
+
+
+# ------------------------------------------------------------------ streaming
+def _state_from_blob(blob, BH, d):
+    hdr = np.frombuffer(blob[:32], np.int32)
+    E = d * d + d
+    s = np.frombuffer(blob[32:32 + 4 * BH * E], np.float32).reshape(BH, E)
+    return int(hdr[2]), s[:, :d * d].reshape(BH, d, d), s[:, d * d:]
+
+
+def _run_stream(w, steps, check_steps=None, rows=None, mask_heads=None, handle=None, start=0, hist=None):
+    mh = w.H if mask_heads is None else mask_heads
+    cfg = hyat.config_from_workload(w, mask_heads=mh)
+    h = hyat.Hyat(cfg) if handle is None else handle
+    L = w.chunk_tokens
+    nwc = w.window_frames // w.chunk_frames
+    kh, vh = hist if hist is not None else ([], [])
+    outs = {}
+    for s in range(start, start + steps):
+        q, k, v, mask = wl.gen_stream_step(w, s)
+        mask = mask[:mh]
+        o = h.stream_step(*_dev(q, k, v), mask=mask)
+        kh.append(k.float().numpy())                    # exact copies of the bf16 values
+        vh.append(v.float().numpy())
+        if check_steps is None or s in check_steps:
+            h.sync()
+            k_all, v_all = np.concatenate(kh, axis=2), np.concatenate(vh, axis=2)
+            ref = oracle.stream_step_attention(f64(q), k_all, v_all, s, L, nwc, mask, rows=rows)
+            got = f64(o) if rows is None else f64(o)[:, :, rows]
+            outs[s] = (got, ref)
+    h.sync()
+    return h, outs, (kh, vh)
+
+
+def test_stream_small_steps_and_state():
+    w = wl.Workload("stream_small", "stream", 1, 2, 128, 200, 24, chunk_frames=3, window_frames=9,
+                    n_steps=8, seed=3)
+    h, outs, (kh, vh) = _run_stream(w, 8)
+    for s, (got, ref) in outs.items():
+        assert_parity("bf16", got, ref, f"step {s}")
+    step, S, z = _state_from_blob(h.get_state(), 2, 128)
+    assert step == 8
+    k_all, v_all = np.concatenate(kh, axis=2), np.concatenate(vh, axis=2)
+    # after step 7 the state holds phi(k) v^T of every chunk evicted up to step 7
+    S_ref, z_ref = oracle.stream_evicted_state(k_all, v_all, 7, w.chunk_tokens, 3)
+    np.testing.assert_allclose(S.reshape(1, 2, 128, 128), S_ref, rtol=0, atol=1e-5 * np.abs(S_ref).max())
+    np.testing.assert_allclose(z.reshape(1, 2, 128), z_ref, rtol=0, atol=1e-5 * np.abs(z_ref).max())
+    h.close()
+
+
+def test_stream_shared_mask_and_f32():
+    w = wl.Workload("stream_f32", "stream", 1, 3, 64, 130, 15, chunk_frames=2, window_frames=4,
+                    n_steps=5, dtype="f32", seed=8)
+    h, outs, _ = _run_stream(w, 5, mask_heads=1)
+    for s, (got, ref) in outs.items():
+        assert_parity("f32", got, ref, f"step {s}")
+    h.close()
+
+
+def test_stream_checkpoint_resume_bit_identical():
+    w = wl.Workload("stream_ckpt", "stream", 1, 2, 128, 200, 30, chunk_frames=3, window_frames=9,
+                    n_steps=10, seed=21)
+    cfg = hyat.config_from_workload(w, mask_heads=2)
+    h1 = hyat.Hyat(cfg)
+    ref_outs = []
+    for s in range(10):
+        q, k, v, mask = wl.gen_stream_step(w, s)
+        ref_outs.append(h1.stream_step(*_dev(q, k, v), mask=mask).cpu())
+        if s == 5:
+            h1.sync()
+            blob = h1.get_state()
+    h1.close()
+    h2 = hyat.Hyat(cfg)
+    h2.set_state(blob)
+    for s in range(6, 10):
+        q, k, v, mask = wl.gen_stream_step(w, s)
+        o = h2.stream_step(*_dev(q, k, v), mask=mask).cpu()
+        assert torch.equal(o, ref_outs[s]), s
+    h2.close()
+
+
+# ------------------------------------------------------------------ errors
+def test_invalid_calls_return_errors_and_handle_stays_usable():
+    w = wl.Workload("err", "stream", 1, 2, 64, 100, 9, chunk_frames=3, window_frames=6, n_steps=2, seed=1)
+    cfg = hyat.config_from_workload(w, mask_heads=1)
+    h = hyat.Hyat(cfg)
+    q, k, v, mask = wl.gen_stream_step(w, 0)
+    bad = mask[:1].copy()
+    bad[0, 0, 0] = 0                                    # diagonal tile dropped
+    with pytest.raises(hyat.HyatError) as ei:
+        h.stream_step(*_dev(q, k, v), mask=bad)
+    assert ei.value.status == hyat.ERR_INVALID_ARG
+    qd, kd, vd = _dev(q, k, v)
+    st = hyat.lib.hyat_fwd_stream_step(h.handle, qd.data_ptr() + 2, kd.data_ptr(), vd.data_ptr(),
+                                       qd.data_ptr(), None, None)
+    assert st == hyat.ERR_INVALID_ARG                   # misaligned pointer
+    st = hyat.lib.hyat_fwd_bidir(h.handle, qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), qd.data_ptr(), None)
+    assert st == hyat.ERR_INVALID_ARG                   # bidirectional call on a stream handle
+    o = h.stream_step(qd, kd, vd, mask=mask[:1])        # still works at step 0
+    h.sync()
+    ref = oracle.stream_step_attention(f64(q), f64(k), f64(v), 0, 300, 2, mask[:1])
+    assert_parity("bf16", f64(o), ref, "after errors")
+    h.close()
+
+
+# ------------------------------------------------------------------ full-size workloads
+def _bidir_sampled(w, heads, per_tile=2, seed=0):
+    o, (q, k, v) = _bidir(w)
+    N = w.N
+    if w.mode == "window":
+        C = w.chunk_tokens
+        tiles = [(c0 + t, min(c0 + t + 128, c0 + C, N)) for c0 in range(0, N, C) for t in (0, 128 * 36)]
+    else:
+        tiles = [(t, min(t + 128, N)) for t in range(0, N, 128 * 97)] + [(N - 96, N)]
+    rows = sample_rows(N, tiles, per_tile=per_tile, seed=seed)
+    qs, ks, vs = q[:, heads], k[:, heads], v[:, heads]
+    if w.mode == "window":
+        ref = _window_ref(w, qs, ks, vs, rows=rows)
+    else:
+        ref = oracle.radial_attention(f64(qs), f64(ks), f64(vs), w.n_frames, w.tokens_per_frame, rows=rows)
+    got = f64(o[:, heads][:, :, rows])
+    return got, ref
+
+
+@pytest.mark.slow
+def test_full_wan13b_bidir_sampled():
+    got, ref = _bidir_sampled(wl.WAN13B_BIDIR, heads=[0, 5, 11])
+    assert_parity("bf16", got, ref, "wan1.3b")
+
+
+@pytest.mark.slow
+def test_full_wan14b_bidir_sampled():
+    got, ref = _bidir_sampled(wl.WAN14B_BIDIR, heads=[0, 17, 39], per_tile=1)
+    assert_parity("bf16", got, ref, "wan14b")
+
+
+@pytest.mark.slow
+def test_full_radial_sampled():
+    got, ref = _bidir_sampled(wl.RADIAL_84F, heads=[0, 11], per_tile=2)
+    assert_parity("bf16", got, ref, "radial")
+
+
+@pytest.mark.slow
+def test_full_stream_sampled():
+    w = wl.STREAM_HF
+    rows = sample_rows(w.chunk_tokens, [(0, 128), (128 * 36, w.chunk_tokens)], per_tile=4,
+                       extra=[1000, 2345, 4000])
+    h, outs, _ = _run_stream(w, w.n_steps, check_steps={0, 1, 2, 3, 4, 17, 39}, rows=rows)
+    for s, (got, ref) in outs.items():
+        assert_parity("bf16", got, ref, f"step {s}")
+    h.close()

@@ -1,0 +1,133 @@
+"""Host-side tests of libhyat (no GPU): exported symbols, layout and eviction
+indexing bit-exact against the oracle's window rules, and argument validation."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from linear_attention_video_hyat_b200 import hyat, workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_library_exports_every_declared_symbol():
+    header = open(os.path.join(ROOT, "include", "hyat.h")).read()
+    declared = sorted(set(re.findall(r"HYAT_API [^;]*?\b(hyat_\w+)\(", header)))
+    assert len(declared) >= 16
+    for name in declared:
+        assert hasattr(hyat.lib, name), name
+    assert sorted(hyat.EXPORTED) == declared
+
+
+def _window_rows_from_layout(work, ent, bh=0):
+    """Map query row -> sorted array of softmax keys, from the C++ layout."""
+    rows = {}
+    for w in work:
+        if w[0] != bh:
+            continue
+        keys = np.concatenate([np.arange(e[0], e[0] + e[1]) for e in ent[w[4]:w[5]]]) \
+            if w[5] > w[4] else np.zeros(0, np.int64)
+        for r in range(w[1], w[1] + w[2]):
+            assert r not in rows
+            rows[r] = keys
+    return rows
+
+
+@pytest.mark.parametrize("T,F,C,h", [(21, 1560, 3, 1), (4, 64, 1, 0), (7, 200, 2, 1), (5, 300, 3, 2),
+                                     (3, 100, 5, 0), (21, 3600, 3, 1)])
+def test_window_layout_matches_oracle(T, F, C, h):
+    cfg = hyat.make_config("window", 1, 2, 128, F, T, C, h)
+    work, ent = hyat.plan_layout(cfg)
+    N = T * F
+    assert set(np.unique(work[:, 0])) == {0, 1}
+    rows = _window_rows_from_layout(work, ent)
+    assert sorted(rows) == list(range(N))
+    sample = np.unique(np.concatenate([np.arange(0, N, max(1, N // 97)), [N - 1]]))
+    soft, lin = oracle.bidir_sets(sample, F, T, C, h)
+    for n, r in enumerate(sample):
+        np.testing.assert_array_equal(rows[r], np.nonzero(soft[n])[0])
+    # every key tile is at most 128 keys, every query tile lies inside one chunk
+    assert np.all((ent[:, 1] >= 1) & (ent[:, 1] <= 128))
+    for w in work:
+        assert (w[1] // F) // C == ((w[1] + w[2] - 1) // F) // C
+
+
+def test_window_layout_tile_counts_wan13b():
+    cfg = hyat.config_from_workload(wl.WAN13B_BIDIR)
+    work, ent = hyat.plan_layout(cfg)
+    assert len(work) == 12 * 7 * 37                     # 37 query tiles per 4680-token chunk
+    per_chunk = [w[5] - w[4] for w in work[:7 * 37:37]]
+    assert per_chunk == [49, 61, 61, 61, 61, 61, 49]    # 6240- and 7800-key windows
+    assert sorted(set(work[:, 2])) == [72, 128]
+
+
+@pytest.mark.parametrize("T,F", [(84, 1560), (12, 300), (9, 100), (5, 64), (7, 130), (1, 50), (21, 3600)])
+def test_radial_mask_bit_exact(T, F):
+    np.testing.assert_array_equal(hyat.radial_mask(T, F), oracle.radial_tile_mask(T, F))
+
+
+def test_radial_layout_counts():
+    cfg = hyat.config_from_workload(wl.RADIAL_84F)
+    work, ent = hyat.plan_layout(cfg)
+    m = oracle.radial_tile_mask(84, 1560)
+    assert len(ent) == int(m.sum()) == 290972
+    for w in work[[0, 1, 500, 1023]]:
+        kt = ent[w[4]:w[5], 0] // 128
+        np.testing.assert_array_equal(kt, np.nonzero(m[w[1] // 128])[0])
+
+
+def test_blockmask_layout_per_head():
+    H, T, F = 3, 5, 100
+    nT = -(-T * F // 128)
+    mask = wl.gen_tile_mask(H, nT, nT, seed=9)
+    cfg = hyat.make_config("blockmask", 2, H, 64, F, T, mask_heads=H)
+    work, ent = hyat.plan_layout(cfg, mask)
+    assert len(work) == 2 * H * nT
+    for w in work:
+        h = w[0] % H
+        soft, _ = oracle.tile_mask_sets(h, [w[1]], mask, T * F)
+        keys = np.concatenate([np.arange(e[0], e[0] + e[1]) for e in ent[w[4]:w[5]]]) \
+            if w[5] > w[4] else np.zeros(0, np.int64)
+        np.testing.assert_array_equal(keys, np.nonzero(soft[0])[0])
+
+
+def test_stream_plan_eviction_indexing():
+    w = wl.STREAM_HF
+    cfg = hyat.config_from_workload(w)
+    nwc = 3
+    slot_of = {}
+    for s in range(w.n_steps):
+        p = hyat.stream_plan(cfg, s)
+        first = max(0, s - nwc + 1)
+        assert p["first_visible"] == first and p["n_visible"] == s - first + 1
+        assert p["evicted"] == (s - nwc if s >= nwc else -1)
+        # the chunk written at step s goes to the slot freed by the evicted chunk
+        if p["evicted"] >= 0:
+            assert slot_of[p["evicted"]] == p["write_slot"]
+        slot_of[s] = p["write_slot"]
+        assert p["slots"] == [slot_of[c] for c in range(first, s + 1)]
+        # evicted frames are exactly the frames the oracle sends to the linear set
+        L = w.chunk_tokens
+        _, lin = oracle.stream_sets(0, [0], s, L, nwc, np.ones((1, 37, 37 * (s - first + 1)), np.uint8))
+        assert int(lin.sum()) == first * L
+
+
+@pytest.mark.parametrize("bad", [dict(d=96), dict(B=0), dict(tokens_per_frame=0), dict(mode=9),
+                                 dict(mode="stream", window_frames=8), dict(mode="blockmask", mask_heads=3),
+                                 dict(dtype=7), dict(scale=-1.0)])
+def test_invalid_configs_rejected(bad):
+    kw = dict(mode="window", B=1, H=2, d=64, tokens_per_frame=64, n_frames=4, chunk_frames=1,
+              window_frames=9)
+    kw.update(bad)
+    if kw["mode"] == "stream":
+        kw["chunk_frames"] = 3
+    cfg = hyat.make_config(**kw)
+    assert hyat.workspace_bytes(cfg) == 0
+
+
+def test_workspace_sizes():
+    for w in (wl.TINY_F32, wl.WAN13B_BIDIR, wl.WAN14B_BIDIR, wl.STREAM_HF, wl.RADIAL_84F):
+        n = hyat.workspace_bytes(hyat.config_from_workload(w))
+        assert 0 < n < 4 << 30, (w.name, n)
