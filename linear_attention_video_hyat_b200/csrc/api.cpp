@@ -21,7 +21,7 @@ enum Kind { K_STATE = 0, K_COMPLEMENT = 1, K_ATTN = 2, K_FOLD = 3, K_PREP = 4 };
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
-  size_t status = 0, work = 0, entries = 0, cm = 0, sseg = 0, srest = 0, srest_t = 0;
+  size_t status = 0, work = 0, entries = 0, pairs = 0, cm = 0, sseg = 0, srest = 0, srest_t = 0;
   size_t ring_k = 0, ring_v = 0, mask = 0, total = 0;
   int64_t n_work = 0, n_entries = 0;
 };
@@ -40,6 +40,7 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
   p.status = take(256);
   p.work = take(sizeof(WorkItem) * std::max<int64_t>(n_work, 1));
   p.entries = take(sizeof(Entry) * std::max<int64_t>(n_entries, 1));
+  p.pairs = take(sizeof(int4) * std::max<int64_t>(n_work, 1));
   if (c.mode == HYAT_MODE_STREAM) {
     const int64_t Lc = stream_chunk_tokens(c), nwc = stream_window_chunks(c), nqt = tiles(Lc);
     p.srest = take(sizeof(float) * BH * E);
@@ -95,6 +96,8 @@ struct hyat_ctx {
   uint32_t* d_status = nullptr;
   WorkItem* d_work = nullptr;
   Entry* d_entries = nullptr;
+  int4* d_pairs = nullptr;
+  int32_t n_pairs = 0;
   float* d_cm = nullptr;
   float* d_sseg = nullptr;
   float* d_srest = nullptr;
@@ -167,6 +170,8 @@ AttnArgs attn_args(hyat_ctx* h, const void* q, const void* k, const void* v, voi
   a.work = h->d_work;
   a.n_work = static_cast<int32_t>(n_work);
   a.entries = h->d_entries;
+  a.pairs = h->d_pairs;
+  a.n_pairs = h->n_pairs;
   a.srest = h->d_srest;
   a.srest_t = h->d_srest_t;
   a.nqg = nqg;
@@ -255,6 +260,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   h->d_status = reinterpret_cast<uint32_t*>(ws + h->plan.status);
   h->d_work = reinterpret_cast<WorkItem*>(ws + h->plan.work);
   h->d_entries = reinterpret_cast<Entry*>(ws + h->plan.entries);
+  h->d_pairs = reinterpret_cast<int4*>(ws + h->plan.pairs);
   h->d_srest = reinterpret_cast<float*>(ws + h->plan.srest);
   h->d_srest_t = reinterpret_cast<uint16_t*>(ws + h->plan.srest_t);
   if (cfg->mode == HYAT_MODE_STREAM) {
@@ -284,6 +290,12 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   if (e == cudaSuccess && !h->lay.entries.empty())
     e = cudaMemcpy(h->d_entries, h->lay.entries.data(), sizeof(Entry) * h->lay.entries.size(),
                    cudaMemcpyHostToDevice);
+  const std::vector<int4> pairs = cfg->mode == HYAT_MODE_STREAM
+                                      ? build_stream_pairs(h->BH, tiles(stream_chunk_tokens(*cfg)))
+                                      : build_pairs(h->lay.work);
+  h->n_pairs = static_cast<int32_t>(pairs.size());
+  if (e == cudaSuccess && !pairs.empty())
+    e = cudaMemcpy(h->d_pairs, pairs.data(), sizeof(int4) * pairs.size(), cudaMemcpyHostToDevice);
   if (e == cudaSuccess && !h->lay.cm.empty())
     e = cudaMemcpy(h->d_cm, h->lay.cm.data(), sizeof(float) * h->lay.cm.size(), cudaMemcpyHostToDevice);
   if (e == cudaSuccess && cfg->mode == HYAT_MODE_STREAM)

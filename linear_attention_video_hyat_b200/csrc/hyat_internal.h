@@ -51,6 +51,10 @@ int32_t tiles(int64_t rows);
 
 // Host layout builders (layout.cpp).
 std::string build_layout(const hyat_config& c, const uint8_t* host_mask, Layout* out);
+// Pair consecutive work items of the same (b, h) into units of two query tiles;
+// `shared` marks pairs whose key lists are identical (loaded once for both).
+std::vector<int4> build_pairs(const std::vector<WorkItem>& work);
+std::vector<int4> build_stream_pairs(int32_t BH, int32_t nqt);
 void radial_tile_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t* out);
 
 // ---- kernel launch wrappers (kernels_simt.cu, attn_tc.cu) ----
@@ -80,6 +84,7 @@ struct AttnArgs {
   int64_t q_rows, k_rows;     // rows per (b, h)
   const WorkItem* work; int32_t n_work;
   const Entry* entries;
+  const int4* pairs; int32_t n_pairs;   // tensor-core path: {item0, item1 or -1, shared list, 0}
   const float* srest;         // [BH][nqg][E]
   const uint16_t* srest_t;    // [BH][nqg][d][d] bf16 (tensor-core path)
   int32_t nqg, d, dtype, BH;

@@ -198,4 +198,27 @@ std::string build_layout(const hyat_config& c, const uint8_t* host_mask, Layout*
   return "unknown mode";
 }
 
+std::vector<int4> build_pairs(const std::vector<WorkItem>& work) {
+  std::vector<int4> pairs;
+  for (size_t i = 0; i < work.size();) {
+    if (i + 1 < work.size() && work[i + 1].bh == work[i].bh) {
+      const bool shared = work[i].entry_begin == work[i + 1].entry_begin && work[i].entry_end == work[i + 1].entry_end;
+      pairs.push_back(make_int4(static_cast<int>(i), static_cast<int>(i + 1), shared ? 1 : 0, 0));
+      i += 2;
+    } else {
+      pairs.push_back(make_int4(static_cast<int>(i), -1, 0, 0));
+      i += 1;
+    }
+  }
+  return pairs;
+}
+
+std::vector<int4> build_stream_pairs(int32_t BH, int32_t nqt) {
+  std::vector<int4> pairs;
+  for (int32_t bh = 0; bh < BH; ++bh)
+    for (int32_t i = 0; i < nqt; i += 2)
+      pairs.push_back(make_int4(bh * nqt + i, i + 1 < nqt ? bh * nqt + i + 1 : -1, 0, 0));
+  return pairs;
+}
+
 }  // namespace hyat
