@@ -127,8 +127,10 @@ __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Smem* sm, u
   }
 }
 
-__device__ __forceinline__ bool aborting(Smem* sm) {
-  return *reinterpret_cast<volatile int32_t*>(&sm->abort_flag) != 0;
+// Warp-uniform bounded wait: every lane waits, and the warp proceeds only if all lanes saw
+// the phase (the TMEM instructions that follow are .sync.aligned).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity, Smem* sm, uint32_t* status) {
+  return __all_sync(0xffffffffu, mbar_wait(b, parity, sm, status));
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
@@ -243,6 +245,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&sm->drain, 1);
     sm->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == MMA_WARP) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm->tmem_base)),
@@ -421,7 +424,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (item < 0) continue;
       const WorkItem wi = p.work[item];
       const int n = wi.entry_end - wi.entry_begin;
-      if (!mbar_wait(&sm->q_full[s], qph, sm, p.status)) break;
+      if (!mbar_wait_warp(&sm->q_full[s], qph, sm, p.status)) break;
       qph ^= 1u;
       // phi(q) of this row -> TMEM (bf16 pairs), l = phi(q) . z
       const float* z = p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D;
@@ -454,7 +457,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       bool ok = true;
       for (int j = 0; j < n; ++j) {
-        if (!mbar_wait(&sm->s_full[s], sph, sm, p.status)) { ok = false; break; }
+        if (!mbar_wait_warp(&sm->s_full[s], sph, sm, p.status)) { ok = false; break; }
         sph ^= 1u;
         tc_fence_after();
         float sv[128];
@@ -480,7 +483,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const float m_new = fmaxf(m, m_cand);
           const float alpha = ex2(m - m_new);
           // the previous P.V (or the linear-branch MMA) must be complete before O is rescaled
-          if (!mbar_wait(&sm->pv_done[s], (pv_phase + j) & 1u, sm, p.status)) { ok = false; break; }
+          if (!mbar_wait_warp(&sm->pv_done[s], (pv_phase + j) & 1u, sm, p.status)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -515,7 +518,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) break;
       // epilogue: o = O / l, bf16, 16-byte stores of the valid rows
-      if (!mbar_wait(&sm->pv_done[s], (pv_phase + n) & 1u, sm, p.status)) break;
+      if (!mbar_wait_warp(&sm->pv_done[s], (pv_phase + n) & 1u, sm, p.status)) break;
       pv_phase += n + 1;
       tc_fence_after();
       const float inv = 1.0f / l;
