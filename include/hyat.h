@@ -178,6 +178,30 @@ HYAT_API hyat_status hyat_stream_set_state(hyat_handle h, const void* src_host, 
 HYAT_API hyat_status hyat_set_profiling(hyat_handle h, int enable);
 HYAT_API hyat_status hyat_kernel_times(hyat_handle h, double* ms, int64_t* launches, int n_kinds);
 
+/* ---- allocation-free forward ----
+ * No passage of the pages corresponds to this entry point; it exists for
+ * callers that cannot allocate device memory where they run the layer (code
+ * running while a caching allocator must not be re-entered, plug-in hosts
+ * whose device memory belongs to another runtime, real-time loops where
+ * cudaMalloc/cudaFree would synchronise the device).
+ *
+ * Same operation and tensor conventions as hyat_fwd_bidir, for WINDOW and
+ * RADIAL configurations, without a handle or a workspace: the scratch lives in
+ * one static 32 MiB __device__ array that every GPU loading the library holds
+ * until the process exits. No cudaMalloc, cudaFree or allocating library call
+ * is made. Returns HYAT_ERR_UNSUPPORTED when the configuration needs more than
+ * 32 MiB of scratch (for example, 12 heads x 21 frames of 1560 tokens at
+ * d = 128 need about 25 MiB), HYAT_ERR_INVALID_ARG for other modes, bad
+ * configurations or pointers that are not 16-byte aligned.
+ * The first call on a device resolves the array's device address; make that
+ * first call before any stream capture. Every call reuses the same array and
+ * leaves the previous call's contents in it (the status word is cleared on
+ * each call): calls that overlap on the GPU -- on different streams, or from
+ * different threads -- race on it and must be serialised by the caller.
+ * Device-side timeouts of this path are not reported (there is no handle). */
+HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, const void* q, const void* k,
+                                            const void* v, void* o, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,153 @@
+// Allocation-free bidirectional forward.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// layer: code that runs while a caching allocator (PyTorch's included) must not
+// be re-entered, plug-in hosts whose memory is owned by another runtime, and
+// real-time loops that forbid cudaMalloc/cudaFree because those calls can
+// synchronise the device and stall for milliseconds. For them this file keeps
+// the forward's scratch (layout tables, per-frame / per-tile linear states,
+// complement states) in one file-scope __device__ array, reserved once per GPU
+// when the library is loaded and held until the process exits. The caller
+// passes only Q, K, V and O.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <vector>
+
+#include "hyat_internal.h"
+
+namespace hyat {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB per GPU
+constexpr int kMaxDevices = 64;
+
+// The scratch. In host code `g_noalloc_scratch` is a host-side stand-in, not a
+// device address: it is never passed to a kernel directly; the device address
+// is obtained with cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+
+// Resolve the scratch address and SM count of the current device (once per device).
+cudaError_t scratch_for_current_device(void** addr, int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+    g_num_sms[dev] = sms;
+  }
+  *addr = g_scratch_addr[dev];
+  *num_sms = g_num_sms[dev];
+  return cudaSuccess;
+}
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+}  // namespace hyat
+
+using namespace hyat;
+
+extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, const void* q, const void* k,
+                                                       const void* v, void* o, void* stream) {
+  if (!cfg || !q || !k || !v || !o) return HYAT_ERR_INVALID_ARG;
+  if (!validate_config(*cfg).empty()) return HYAT_ERR_INVALID_ARG;
+  if (cfg->mode != HYAT_MODE_WINDOW && cfg->mode != HYAT_MODE_RADIAL) return HYAT_ERR_INVALID_ARG;
+  for (const void* p : {q, k, v, static_cast<const void*>(o)})
+    if (reinterpret_cast<uintptr_t>(p) & 15u) return HYAT_ERR_INVALID_ARG;
+
+  Layout L;
+  if (!build_layout(*cfg, nullptr, &L).empty()) return HYAT_ERR_INVALID_ARG;
+  const std::vector<int4> pairs = build_pairs(L.work);
+  const int64_t BH = int64_t(cfg->B) * cfg->H;
+  const int64_t E = int64_t(cfg->d) * cfg->d + cfg->d;
+  const int64_t rows = rows_q(*cfg);
+
+  // carve the static scratch
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o2 = off; off = up256(off + bytes); return o2; };
+  const size_t o_status = take(256);
+  const size_t o_work = take(sizeof(WorkItem) * L.work.size());
+  const size_t o_entries = take(sizeof(Entry) * (L.entries.empty() ? 1 : L.entries.size()));
+  const size_t o_pairs = take(sizeof(int4) * pairs.size());
+  const size_t o_cm = take(sizeof(float) * L.cm.size());
+  const size_t o_sseg = take(sizeof(float) * size_t(BH) * L.nseg * E);
+  const size_t o_srest = take(sizeof(float) * size_t(BH) * L.nqg * E);
+  const size_t o_srest_t = take(2 * size_t(BH) * L.nqg * cfg->d * cfg->d);
+  if (off > kNoAllocScratchBytes) return HYAT_ERR_UNSUPPORTED;  // needs more than the static scratch
+
+  void* base = nullptr;
+  int num_sms = 0;
+  if (scratch_for_current_device(&base, &num_sms) != cudaSuccess) return HYAT_ERR_CUDA;
+  char* ws = static_cast<char*>(base);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // layout tables: pageable host -> scratch (the copy has consumed the vectors when it returns);
+  // the status word starts at zero on every call
+  cudaError_t e = cudaMemsetAsync(ws + o_status, 0, 256, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + o_work, L.work.data(), sizeof(WorkItem) * L.work.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !L.entries.empty())
+    e = cudaMemcpyAsync(ws + o_entries, L.entries.data(), sizeof(Entry) * L.entries.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(ws + o_pairs, pairs.data(), sizeof(int4) * pairs.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(ws + o_cm, L.cm.data(), sizeof(float) * L.cm.size(), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return HYAT_ERR_CUDA;
+
+  SegStateArgs sa{};
+  sa.k = k; sa.v = v; sa.rows_per_bh = rows;
+  sa.BH = static_cast<int32_t>(BH); sa.d = cfg->d; sa.dtype = cfg->dtype;
+  sa.nseg = L.nseg; sa.seg_base = 0; sa.seg_stride = L.seg_stride; sa.seg_len = L.seg_len;
+  sa.out = reinterpret_cast<float*>(ws + o_sseg); sa.accumulate = 0;
+  if (launch_seg_state(sa, s) != cudaSuccess) return HYAT_ERR_CUDA;
+
+  ComplementArgs ca{};
+  ca.sseg = sa.out; ca.cm = reinterpret_cast<const float*>(ws + o_cm);
+  ca.srest = reinterpret_cast<float*>(ws + o_srest);
+  ca.BH = static_cast<int32_t>(BH); ca.H = cfg->H; ca.cm_heads = L.cm_heads; ca.nseg = L.nseg; ca.nqg = L.nqg;
+  ca.E = static_cast<int32_t>(E);
+  if (launch_complement(ca, s) != cudaSuccess) return HYAT_ERR_CUDA;
+
+  AttnArgs a{};
+  a.q = q; a.k = k; a.v = v; a.o = o;
+  a.q_rows = rows; a.k_rows = rows;
+  a.work = reinterpret_cast<const WorkItem*>(ws + o_work);
+  a.n_work = static_cast<int32_t>(L.work.size());
+  a.entries = reinterpret_cast<const Entry*>(ws + o_entries);
+  a.pairs = reinterpret_cast<const int4*>(ws + o_pairs);
+  a.n_pairs = static_cast<int32_t>(pairs.size());
+  a.srest = ca.srest;
+  a.srest_t = reinterpret_cast<const uint16_t*>(ws + o_srest_t);
+  a.nqg = L.nqg; a.d = cfg->d; a.dtype = cfg->dtype; a.BH = static_cast<int32_t>(BH);
+  const float scale = cfg->scale > 0.0f ? cfg->scale : 1.0f / sqrtf(float(cfg->d));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.status = reinterpret_cast<uint32_t*>(ws + o_status);
+
+  int major = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return HYAT_ERR_CUDA;
+  const bool use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
+                      attn_tc_supported(cfg->d, cfg->dtype);
+  if (use_tc) {
+    if (launch_state_transpose_bf16(ca.srest, reinterpret_cast<uint16_t*>(ws + o_srest_t), BH * L.nqg, cfg->d, s) !=
+        cudaSuccess)
+      return HYAT_ERR_CUDA;
+    if (launch_attn_tc(a, num_sms, s) != cudaSuccess) return HYAT_ERR_CUDA;
+  } else {
+    if (launch_attn_simt(a, s) != cudaSuccess) return HYAT_ERR_CUDA;
+  }
+  return HYAT_OK;
+}

@@ -30,7 +30,7 @@ EXPORTED = (
     "hyat_workspace_bytes", "hyat_create", "hyat_fwd_bidir", "hyat_fwd_stream_step", "hyat_sync",
     "hyat_destroy", "hyat_last_error", "hyat_status_string", "hyat_plan_layout", "hyat_radial_mask",
     "hyat_stream_plan", "hyat_stream_state_bytes", "hyat_stream_get_state", "hyat_stream_set_state",
-    "hyat_set_profiling", "hyat_kernel_times",
+    "hyat_set_profiling", "hyat_kernel_times", "hyat_fwd_bidir_noalloc",
 )
 
 
@@ -75,6 +75,7 @@ def _load():
         "hyat_stream_set_state": (ctypes.c_int, [P, P, S]),
         "hyat_set_profiling": (ctypes.c_int, [P, ctypes.c_int]),
         "hyat_kernel_times": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64), ctypes.c_int]),
+        "hyat_fwd_bidir_noalloc": (ctypes.c_int, [CP, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
