@@ -333,8 +333,10 @@ hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const vo
   sa.k = k; sa.v = v; sa.rows_per_bh = h->rk;
   sa.BH = h->BH; sa.d = h->cfg.d; sa.dtype = h->cfg.dtype;
   sa.nseg = L.nseg; sa.seg_base = 0; sa.seg_stride = L.seg_stride; sa.seg_len = L.seg_len;
-  sa.out = h->d_sseg; sa.accumulate = 0;
-  cudaError_t e = timed(h, K_STATE, s, [&] { return launch_seg_state(sa, s); });
+  sa.out = h->d_sseg; sa.accumulate = 0; sa.status = h->d_status;
+  cudaError_t e = timed(h, K_STATE, s, [&] {
+    return h->use_tc ? launch_seg_state_tc(sa, h->num_sms, s) : launch_seg_state(sa, s);
+  });
   if (e != cudaSuccess) return cuda_fail(h, e, "segment state kernel");
   ComplementArgs ca{};
   ca.sseg = h->d_sseg; ca.cm = h->d_cm; ca.srest = h->d_srest;
@@ -378,8 +380,8 @@ hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, co
       sa.k = h->d_ring_k; sa.v = h->d_ring_v; sa.rows_per_bh = h->rk;
       sa.BH = h->BH; sa.d = c.d; sa.dtype = c.dtype;
       sa.nseg = 1; sa.seg_base = slot * Lc; sa.seg_stride = Lc; sa.seg_len = Lc;
-      sa.out = h->d_srest; sa.accumulate = 1;
-      cudaError_t e2 = launch_seg_state(sa, s);
+      sa.out = h->d_srest; sa.accumulate = 1; sa.status = h->d_status;
+      cudaError_t e2 = h->use_tc ? launch_seg_state_tc(sa, h->num_sms, s) : launch_seg_state(sa, s);
       if (e2 != cudaSuccess) return e2;
     }
     RingCopyArgs ra{};

@@ -32,19 +32,29 @@
 #include <cstring>
 
 #include "hyat_internal.h"
+#include "tc_common.cuh"
 
 namespace hyat {
 namespace {
 
-constexpr int D = 128;
-constexpr int TILE_BYTES = 128 * D * 2;          // one 128 x 128 bf16 tile
-constexpr int HALF_BYTES = TILE_BYTES / 2;       // 64 columns (128 B rows)
+using namespace tc;
 constexpr int NS = 5;                            // K/V stage ring
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 384;                 // 3 warpgroups
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
+// Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); warpgroup 2
+// (TMA, MMA, 2 idle warps) drops to 88, the two softmax warpgroups rise to 208:
+// 8 warps x 32 x 208 + 4 warps x 32 x 88 = 64512. Per SM sub-partition: 2 softmax warps
+// and 1 warp of group 2 = 2 x 32 x 208 + 32 x 88 = 16128 <= 16384.
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsLoadMma = 88;
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
-constexpr unsigned long long kTimeoutNs = 2000000000ull;
+// Of every 8 score pairs of a full tile, this many take exp2 on the FMA pipe (exp2_fma) and
+// the rest on MUFU, so the two pipes share the exponentials; partial tiles use MUFU only.
+#ifndef HYAT_EMU_OF8
+#define HYAT_EMU_OF8 0
+#endif
+constexpr int kEmuOf8 = HYAT_EMU_OF8;
 
 // instruction descriptor, kind::f16: D f32, A/B bf16, M = 128, N = 128
 constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -75,43 +85,8 @@ struct TcParams {
   uint32_t* status;
 };
 
-// ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait on a phase parity. Returns false if the kernel is aborting.
-__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Smem* sm, uint32_t* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Smem* sm, uint32_t* status) {
   if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
@@ -133,92 +108,178 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity, Sme
   return __all_sync(0xffffffffu, mbar_wait(b, parity, sm, status));
 }
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int x, int y, int z, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
+// ------------------------------------------------------------------ softmax role
+// Warp-uniform wait with an inline fast path.
+__device__ __forceinline__ bool wait_warp(uint64_t* b, uint32_t parity, Smem* sm, uint32_t* status) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(b, parity))) return true;
+  return mbar_wait_warp(b, parity, sm, status);
 }
 
-// a 128-row x 128-column bf16 tile = two boxes of 64 columns (128-byte rows)
-__device__ __forceinline__ void tma_tile(uint8_t* dst, const CUtensorMap* tm, int row, int z, uint64_t* bar) {
-  mbar_expect_tx(bar, TILE_BYTES);
-  tma_load_3d(smem_u32(dst), tm, 0, row, z, bar);
-  tma_load_3d(smem_u32(dst + HALF_BYTES), tm, 64, row, z, bar);
-}
-
-// shared-memory matrix descriptor, 128-byte swizzle, sm100 version bits
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// K-major operand (rows = M or N, 128 columns of K in two 64-column halves); K step kk of 16
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk) {
-  return sdesc(base + (kk >> 2) * HALF_BYTES + (kk & 3) * 32, 16, 1024);
-}
-// MN-major operand (rows = K, 128 columns of N in two 64-column halves); K step kk of 16 rows
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int kk) {
-  return sdesc(base + kk * 2048, HALF_BYTES, 1024);
-}
-
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-#define HYAT_R8(i) "=r"(r[i + 0]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
-#define HYAT_W8(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
-
-// 32 consecutive 32-bit columns of this thread's TMEM lane
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : HYAT_R8(0), HYAT_R8(8), HYAT_R8(16), HYAT_R8(24)
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      HYAT_W8(0), HYAT_W8(8), HYAT_W8(16), HYAT_W8(24)
-      : "memory");
-}
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ float phi_elu1(float x) {
-  return x > 0.0f ? x + 1.0f : ex2(x * 1.4426950408889634f);
+// One query row per thread (TMEM lane = row). Slot s = warpgroup index.
+__device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32_t tmem, int warp) {
+  const int s = warp >> 2;
+  const int row = threadIdx.x & 127;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t tS = tmem + s * 128 + lane_off;
+  const uint32_t tO = tmem + 256 + s * 128 + lane_off;
+  uint64_t* q_full = &sm->q_full[s];
+  uint64_t* s_full = &sm->s_full[s];
+  uint64_t* p_full = &sm->p_full[s];
+  uint64_t* pv_done = &sm->pv_done[s];
+  const float sl = p.scale_log2;
+  uint32_t qph = 0, sph = 0;
+  uint32_t pv_phase = 0;                            // pv_done phases completed before this pair
+  for (int pi = blockIdx.x; pi < p.n_pairs; pi += gridDim.x) {
+    const int4 pr = p.pairs[pi];
+    const int item = s == 0 ? pr.x : pr.y;
+    if (item < 0) continue;
+    const WorkItem wi = p.work[item];
+    const int n = wi.entry_end - wi.entry_begin;
+    const Entry* ent = p.entries + wi.entry_begin;
+    int klen_next = n > 0 ? ent[0].k_len : 128;
+    if (!wait_warp(q_full, qph, sm, p.status)) return;
+    qph ^= 1u;
+    // phi(q) of this row -> TMEM (bf16 pairs), l = phi(q) . z
+    const float* z = p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D;
+    float l = 0.0f, m = 0.0f;
+    {
+      const uint8_t* qrow = sm->q[s] + row * 128;
+      float lz[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int c = 0; c < 16; ++c) {            // 8 columns per step
+        const uint4 raw = *reinterpret_cast<const uint4*>(qrow + (c >> 3) * HALF_BYTES + (((c & 7) ^ (row & 7)) << 4));
+        const float4 za = __ldg(reinterpret_cast<const float4*>(z + 8 * c));
+        const float4 zb = __ldg(reinterpret_cast<const float4*>(z + 8 * c + 4));
+        const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+          const float f0 = phi_elu1(f.x), f1 = phi_elu1(f.y);
+          lz[e] = fmaf(f0, zz[2 * e], lz[e]);
+          lz[e] = fmaf(f1, zz[2 * e + 1], lz[e]);
+          pk[e] = pack_bf16(f0, f1);
+        }
+        tmem_st4(tS + 4 * c, pk);
+      }
+      l = (lz[0] + lz[1]) + (lz[2] + lz[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    for (int j = 0; j < n; ++j) {
+      const int klen = klen_next;
+      if (j + 1 < n) klen_next = ent[j + 1].k_len;
+      if (!wait_warp(s_full, sph, sm, p.status)) return;
+      sph ^= 1u;
+      tc_fence_after();
+      uint32_t r[128];
+      tmem_ld32p(tS, r);
+      tmem_ld32p(tS + 32, r + 32);
+      tmem_ld32p(tS + 64, r + 64);
+      tmem_ld32p(tS + 96, r + 96);
+      tmem_wait_ld();
+      if (klen < 128) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) r[i] = i < klen ? r[i] : 0xff800000u;   // -inf
+      }
+      // row max: 8 independent chains of 3-input max, then a short tree
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float a = fmax3(u2f(r[k]), u2f(r[k + 8]), u2f(r[k + 16]));
+#pragma unroll
+        for (int t = 3; t < 15; t += 2) a = fmax3(a, u2f(r[k + 8 * t]), u2f(r[k + 8 * t + 8]));
+        mx[k] = fmaxf(a, u2f(r[k + 120]));
+      }
+      const float mrow = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+      const float m_cand = mrow * sl;
+      if (__any_sync(0xffffffffu, m_cand > m + kRescaleThreshold)) {
+        const float m_new = fmaxf(m, m_cand);
+        const float alpha = ex2(m - m_new);
+        // the previous P.V (or the linear-branch MMA) must be complete before O is rescaled
+        if (!wait_warp(pv_done, (pv_phase + j) & 1u, sm, p.status)) return;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(u2f(o[i]) * alpha);
+          tmem_st32(tO + c * 32, o);
+        }
+        tmem_wait_st();
+        l *= alpha;
+        m = m_new;
+      }
+      const float neg_m = -m;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (kEmuOf8 > 0 && klen == 128) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x0 = fmaf(u2f(r[h * 64 + 2 * i]), sl, neg_m);
+            const float x1 = fmaf(u2f(r[h * 64 + 2 * i + 1]), sl, neg_m);
+            const bool emu = (i & 7) < kEmuOf8;
+            const float p0 = emu ? exp2_fma(x0) : ex2(x0);
+            const float p1 = emu ? exp2_fma(x1) : ex2(x1);
+            acc[(2 * i) & 7] += p0;
+            acc[(2 * i + 1) & 7] += p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st32(tS + h * 32, pk);
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2(fmaf(u2f(r[h * 64 + 2 * i]), sl, neg_m));
+            const float p1 = ex2(fmaf(u2f(r[h * 64 + 2 * i + 1]), sl, neg_m));
+            acc[(2 * i) & 7] += p0;
+            acc[(2 * i + 1) & 7] += p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st32(tS + h * 32, pk);
+        }
+      }
+      l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // epilogue: o = O / l, bf16, 16-byte stores of the valid rows
+    if (!wait_warp(pv_done, (pv_phase + n) & 1u, sm, p.status)) return;
+    pv_phase += n + 1;
+    tc_fence_after();
+    const float inv = 1.0f / l;
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
+                                          (static_cast<int64_t>(wi.bh) * p.q_rows + wi.q_row + row) * D);
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      uint32_t r[64];
+      tmem_ld32p(tO + h * 64, r);
+      tmem_ld32p(tO + h * 64 + 32, r + 32);
+      tmem_wait_ld();
+      if (row < wi.q_len) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 w;
+          w.x = pack_bf16(u2f(r[8 * v + 0]) * inv, u2f(r[8 * v + 1]) * inv);
+          w.y = pack_bf16(u2f(r[8 * v + 2]) * inv, u2f(r[8 * v + 3]) * inv);
+          w.z = pack_bf16(u2f(r[8 * v + 4]) * inv, u2f(r[8 * v + 5]) * inv);
+          w.w = pack_bf16(u2f(r[8 * v + 6]) * inv, u2f(r[8 * v + 7]) * inv);
+          dst[h * 8 + v] = w;
+        }
+      }
+    }
+    tc_fence_before();
+  }
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -257,51 +318,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
 
-  if (warp == PRODUCER_WARP) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ producer
+  if (warp >= 8) {
+    // ------------------------------------------------------------ warpgroup 2: TMA + MMA
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLoadMma));
+    if (warp == PRODUCER_WARP && lane == 0) {
       int st = 0;
-      uint32_t ph = 0;
-      uint32_t qph[2] = {0, 0};
-      uint32_t pending = 0;               // stages holding a load not yet seen complete
-      uint32_t pending_ph[NS];
+      uint32_t ph = 0, qph0 = 0, qph1 = 0;
+      uint32_t pending = 0, pending_ph = 0;   // stages with a load in flight, and its phase bit
       bool ok = true;
       auto take = [&](const CUtensorMap* tm, int row, int z) -> bool {
         if (!mbar_wait(&sm->kv_empty[st], ph ^ 1u, sm, p.status)) return false;
         tma_tile(sm->kv[st], tm, row, z, &sm->kv_full[st]);
         pending |= 1u << st;
-        pending_ph[st] = ph;
+        pending_ph = (pending_ph & ~(1u << st)) | (ph << st);
         if (++st == NS) { st = 0; ph ^= 1u; }
         return true;
       };
       for (int pi = blockIdx.x; pi < p.n_pairs && ok; pi += gridDim.x) {
         const int4 pr = p.pairs[pi];
-        const int items[2] = {pr.x, pr.y};
-        const bool shared = pr.z != 0;
-        WorkItem wi[2];
-        int n[2] = {0, 0};
-        for (int s = 0; s < 2; ++s) {
-          if (items[s] < 0) continue;
-          wi[s] = p.work[items[s]];
-          n[s] = wi[s].entry_end - wi[s].entry_begin;
-          if (!mbar_wait(&sm->q_empty[s], qph[s] ^ 1u, sm, p.status)) { ok = false; break; }
-          qph[s] ^= 1u;
-          tma_tile(sm->q[s], &tmQ, wi[s].q_row, wi[s].bh, &sm->q_full[s]);
-        }
+        const bool has1 = pr.y >= 0, shared = pr.z != 0;
+        const WorkItem w0 = p.work[pr.x];
+        WorkItem w1 = w0;
+        if (has1) w1 = p.work[pr.y];
+        const int n0 = w0.entry_end - w0.entry_begin;
+        const int n1 = has1 ? w1.entry_end - w1.entry_begin : 0;
+        const Entry* e0 = p.entries + w0.entry_begin;
+        const Entry* e1 = p.entries + w1.entry_begin;
+        ok = mbar_wait(&sm->q_empty[0], qph0 ^ 1u, sm, p.status);
         if (!ok) break;
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (items[s] < 0) continue;
-          ok = take(&tmS, 0, wi[s].bh * p.nqg + wi[s].state_group);
-          if (ok && n[s] > 0 && (s == 0 || !shared))
-            ok = take(&tmK, p.entries[wi[s].entry_begin].k_row, wi[s].bh);
+        qph0 ^= 1u;
+        tma_tile(sm->q[0], &tmQ, w0.q_row, w0.bh, &sm->q_full[0]);
+        if (has1) {
+          ok = mbar_wait(&sm->q_empty[1], qph1 ^ 1u, sm, p.status);
+          if (!ok) break;
+          qph1 ^= 1u;
+          tma_tile(sm->q[1], &tmQ, w1.q_row, w1.bh, &sm->q_full[1]);
         }
-        const int nmax = n[0] > n[1] ? n[0] : n[1];
+        ok = take(&tmS, 0, w0.bh * p.nqg + w0.state_group);
+        if (ok && n0 > 0) ok = take(&tmK, e0[0].k_row, w0.bh);
+        if (ok && has1) {
+          ok = take(&tmS, 0, w1.bh * p.nqg + w1.state_group);
+          if (ok && n1 > 0 && !shared) ok = take(&tmK, e1[0].k_row, w1.bh);
+        }
+        const int nmax = n0 > n1 ? n0 : n1;
         for (int j = 0; j < nmax && ok; ++j) {
-          for (int s = 0; s < 2 && ok; ++s) {
-            if (items[s] < 0 || j >= n[s] || (s == 1 && shared)) continue;
-            const Entry* e = p.entries + wi[s].entry_begin;
-            ok = take(&tmV, e[j].k_row, wi[s].bh);
-            if (ok && j + 1 < n[s]) ok = take(&tmK, e[j + 1].k_row, wi[s].bh);
+          if (j < n0) {
+            ok = take(&tmV, e0[j].k_row, w0.bh);
+            if (ok && j + 1 < n0) ok = take(&tmK, e0[j + 1].k_row, w0.bh);
+          }
+          if (ok && has1 && !shared && j < n1) {
+            ok = take(&tmV, e1[j].k_row, w1.bh);
+            if (ok && j + 1 < n1) ok = take(&tmK, e1[j + 1].k_row, w1.bh);
           }
         }
       }
@@ -310,95 +377,111 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int i = 0; i < NS; ++i) {
           if (!(pending & (1u << i))) continue;
           const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(&sm->kv_full[i], pending_ph[i]) && globaltimer() - t0 < kTimeoutNs) {
+          while (!mbar_try_wait(&sm->kv_full[i], (pending_ph >> i) & 1u) && globaltimer() - t0 < kTimeoutNs) {
           }
         }
       }
-    }
-  } else if (warp == MMA_WARP) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
+    } else if (warp == MMA_WARP && lane == 0) {
       int st = 0;
-      uint32_t ph = 0;
-      uint32_t qph[2] = {0, 0}, pph[2] = {0, 0};
+      uint32_t ph = 0, qph0 = 0, qph1 = 0, pph0 = 0, pph1 = 0;
       bool ok = true;
-      const uint32_t tS[2] = {tmem, tmem + 128};
-      const uint32_t tO[2] = {tmem + 256, tmem + 384};
-      auto next_stage = [&](int* out) -> bool {
+      auto next_stage = [&](int& out) -> bool {
         if (!mbar_wait(&sm->kv_full[st], ph, sm, p.status)) return false;
         tc_fence_after();
-        *out = st;
+        out = st;
         if (++st == NS) { st = 0; ph ^= 1u; }
         return true;
       };
-      auto wait_p = [&](int s) -> bool {
-        if (!mbar_wait(&sm->p_full[s], pph[s], sm, p.status)) return false;
-        pph[s] ^= 1u;
+      auto wait_p = [&](uint64_t* bar, uint32_t& phase) -> bool {
+        if (!mbar_wait(bar, phase, sm, p.status)) return false;
+        phase ^= 1u;
         tc_fence_after();
         return true;
       };
-      auto qk = [&](int s, int stage) {
-        const uint32_t qa = smem_u32(sm->q[s]), kb = smem_u32(sm->kv[stage]);
+      auto qk = [&](uint32_t tS, const uint8_t* qbuf, int stage, uint64_t* done) {
+        const uint32_t qa = smem_u32(qbuf), kb = smem_u32(sm->kv[stage]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tS[s], desc_kmajor(qa, kk), desc_kmajor(kb, kk), kIdescKK, kk > 0);
-        mma_commit(&sm->s_full[s]);
+        for (int kk = 0; kk < 8; ++kk) mma_ss(tS, desc_kmajor(qa, kk), desc_kmajor(kb, kk), kIdescKK, kk > 0);
+        mma_commit(done);
       };
-      auto pv = [&](int s, int stage) {
+      auto pv = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
         const uint32_t vb = smem_u32(sm->kv[stage]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts(tO[s], tS[s] + kk * 8, desc_mnmajor(vb, kk), kIdescKMN, 1);
-        mma_commit(&sm->pv_done[s]);
+        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, desc_mnmajor(vb, kk), kIdescKMN, 1);
+        mma_commit(done);
       };
+      auto linear = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
+        const uint32_t sb = smem_u32(sm->kv[stage]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, desc_kmajor(sb, kk), kIdescKK, kk > 0);
+        mma_commit(done);
+      };
+      const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
       for (int pi = blockIdx.x; pi < p.n_pairs && ok; pi += gridDim.x) {
         const int4 pr = p.pairs[pi];
-        const int items[2] = {pr.x, pr.y};
-        const bool shared = pr.z != 0;
-        int n[2] = {0, 0};
-        for (int s = 0; s < 2; ++s)
-          if (items[s] >= 0) n[s] = p.work[items[s]].entry_end - p.work[items[s]].entry_begin;
-        int kst[2] = {-1, -1};
-        // linear branch: O_s = phi(Q_s) S_rest^T, then the first QK
-        for (int s = 0; s < 2 && ok; ++s) {
-          if (items[s] < 0) continue;
-          int sst;
-          ok = wait_p(s) && next_stage(&sst);
+        const bool has1 = pr.y >= 0, shared = pr.z != 0;
+        const int n0 = p.work[pr.x].entry_end - p.work[pr.x].entry_begin;
+        const int n1 = has1 ? p.work[pr.y].entry_end - p.work[pr.y].entry_begin : 0;
+        int k0 = -1, k1 = -1, v0 = -1, v1 = -1, sst = -1;
+        // slot 0: O0 = phi(Q0) S_rest^T, then S0 = Q0 K^T
+        ok = wait_p(&sm->p_full[0], pph0) && next_stage(sst);
+        if (!ok) break;
+        linear(tO0, tS0, sst, &sm->pv_done[0]);
+        mma_commit(&sm->kv_empty[sst]);
+        ok = mbar_wait(&sm->q_full[0], qph0, sm, p.status);
+        if (!ok) break;
+        qph0 ^= 1u;
+        tc_fence_after();
+        if (n0 > 0) {
+          ok = next_stage(k0);
           if (!ok) break;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_ts(tO[s], tS[s] + kk * 8, desc_kmajor(smem_u32(sm->kv[sst]), kk), kIdescKK, kk > 0);
-          mma_commit(&sm->pv_done[s]);
-          mma_commit(&sm->kv_empty[sst]);
-          if (n[s] > 0) {
-            if (!mbar_wait(&sm->q_full[s], qph[s], sm, p.status)) { ok = false; break; }
-            tc_fence_after();
-            if (s == 1 && shared) kst[1] = kst[0];
-            else if (!next_stage(&kst[s])) { ok = false; break; }
-            qk(s, kst[s]);
-            if (!(s == 0 && shared)) mma_commit(&sm->kv_empty[kst[s]]);
-            if (n[s] == 1) mma_commit(&sm->q_empty[s]);
-          } else {
-            if (!mbar_wait(&sm->q_full[s], qph[s], sm, p.status)) { ok = false; break; }
-            mma_commit(&sm->q_empty[s]);
-          }
-          qph[s] ^= 1u;
+          qk(tS0, sm->q[0], k0, &sm->s_full[0]);
+          if (!shared) mma_commit(&sm->kv_empty[k0]);
         }
-        const int nmax = n[0] > n[1] ? n[0] : n[1];
-        int vst0 = -1;
+        if (n0 <= 1) mma_commit(&sm->q_empty[0]);
+        // slot 1
+        if (has1) {
+          ok = wait_p(&sm->p_full[1], pph1) && next_stage(sst);
+          if (!ok) break;
+          linear(tO1, tS1, sst, &sm->pv_done[1]);
+          mma_commit(&sm->kv_empty[sst]);
+          ok = mbar_wait(&sm->q_full[1], qph1, sm, p.status);
+          if (!ok) break;
+          qph1 ^= 1u;
+          tc_fence_after();
+          if (n1 > 0) {
+            if (shared) k1 = k0;
+            else if (!(ok = next_stage(k1))) break;
+            qk(tS1, sm->q[1], k1, &sm->s_full[1]);
+            mma_commit(&sm->kv_empty[k1]);
+          }
+          if (n1 <= 1) mma_commit(&sm->q_empty[1]);
+        }
+        const int nmax = n0 > n1 ? n0 : n1;
         for (int j = 0; j < nmax && ok; ++j) {
-          for (int s = 0; s < 2 && ok; ++s) {
-            if (items[s] < 0 || j >= n[s]) continue;
-            int vst;
-            if (!wait_p(s)) { ok = false; break; }
-            if (s == 1 && shared) vst = vst0;
-            else if (!next_stage(&vst)) { ok = false; break; }
-            if (s == 0) vst0 = vst;
-            pv(s, vst);
-            if (!(s == 0 && shared)) mma_commit(&sm->kv_empty[vst]);
-            if (j + 1 < n[s]) {
-              if (s == 1 && shared) kst[1] = kst[0];
-              else if (!next_stage(&kst[s])) { ok = false; break; }
-              qk(s, kst[s]);
-              if (!(s == 0 && shared)) mma_commit(&sm->kv_empty[kst[s]]);
-              if (j + 2 == n[s]) mma_commit(&sm->q_empty[s]);
+          if (j < n0) {
+            if (!(ok = wait_p(&sm->p_full[0], pph0) && next_stage(v0))) break;
+            pv(tO0, tS0, v0, &sm->pv_done[0]);
+            if (!shared) mma_commit(&sm->kv_empty[v0]);
+            if (j + 1 < n0) {
+              if (!(ok = next_stage(k0))) break;
+              qk(tS0, sm->q[0], k0, &sm->s_full[0]);
+              if (!shared) mma_commit(&sm->kv_empty[k0]);
+              if (j + 2 == n0) mma_commit(&sm->q_empty[0]);
+            }
+          }
+          if (has1 && j < n1) {
+            if (!(ok = wait_p(&sm->p_full[1], pph1))) break;
+            if (shared) v1 = v0;
+            else if (!(ok = next_stage(v1))) break;
+            pv(tO1, tS1, v1, &sm->pv_done[1]);
+            mma_commit(&sm->kv_empty[v1]);
+            if (j + 1 < n1) {
+              if (shared) k1 = k0;
+              else if (!(ok = next_stage(k1))) break;
+              qk(tS1, sm->q[1], k1, &sm->s_full[1]);
+              mma_commit(&sm->kv_empty[k1]);
+              if (j + 2 == n1) mma_commit(&sm->q_empty[1]);
             }
           }
         }
@@ -410,139 +493,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
-    // -------------------------------------------------------------- softmax
-    const int s = warp >> 2;                          // slot of this warpgroup
-    const int row = threadIdx.x & 127;                // query row in the tile = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + s * 128 + lane_off;
-    const uint32_t tO = tmem + 256 + s * 128 + lane_off;
-    uint32_t qph = 0, sph = 0;
-    uint32_t pv_phase = 0;                            // pv_done phases completed before this pair
-    for (int pi = blockIdx.x; pi < p.n_pairs; pi += gridDim.x) {
-      const int4 pr = p.pairs[pi];
-      const int item = s == 0 ? pr.x : pr.y;
-      if (item < 0) continue;
-      const WorkItem wi = p.work[item];
-      const int n = wi.entry_end - wi.entry_begin;
-      if (!mbar_wait_warp(&sm->q_full[s], qph, sm, p.status)) break;
-      qph ^= 1u;
-      // phi(q) of this row -> TMEM (bf16 pairs), l = phi(q) . z
-      const float* z = p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D;
-      float l = 0.0f, m = 0.0f;
-      {
-        const uint8_t* qrow = sm->q[s] + row * 128;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t packed[32];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(qrow + half * HALF_BYTES + ((c ^ (row & 7)) << 4));
-            const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w4[e]);
-              const float2 f = __bfloat1622float2(b2);
-              const float f0 = phi_elu1(f.x), f1 = phi_elu1(f.y);
-              const int col = half * 64 + c * 8 + e * 2;
-              l = fmaf(f0, __ldg(z + col), l);
-              l = fmaf(f1, __ldg(z + col + 1), l);
-              packed[c * 4 + e] = pack_bf16(f0, f1);
-            }
-          }
-          tmem_st32(tS + half * 32, packed);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&sm->p_full[s]);
-      }
-      bool ok = true;
-      for (int j = 0; j < n; ++j) {
-        if (!mbar_wait_warp(&sm->s_full[s], sph, sm, p.status)) { ok = false; break; }
-        sph ^= 1u;
-        tc_fence_after();
-        float sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tS + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
-        }
-        const int klen = p.entries[wi.entry_begin + j].k_len;
-        if (klen < 128) {
-#pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i >= klen) sv[i] = -INFINITY;
-        }
-        float mx = sv[0];
-#pragma unroll
-        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, sv[i]);
-        const float m_cand = mx * p.scale_log2;
-        if (__any_sync(0xffffffffu, m_cand > m + kRescaleThreshold)) {
-          const float m_new = fmaxf(m, m_cand);
-          const float alpha = ex2(m - m_new);
-          // the previous P.V (or the linear-branch MMA) must be complete before O is rescaled
-          if (!mbar_wait_warp(&sm->pv_done[s], (pv_phase + j) & 1u, sm, p.status)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + c * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tO + c * 32, r);
-          }
-          tmem_wait_st();
-          l *= alpha;
-          m = m_new;
-        }
-        float rs = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t packed[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2(fmaf(sv[c * 64 + 2 * i], p.scale_log2, -m));
-            const float p1 = ex2(fmaf(sv[c * 64 + 2 * i + 1], p.scale_log2, -m));
-            rs += p0 + p1;
-            packed[i] = pack_bf16(p0, p1);
-          }
-          tmem_st32(tS + c * 32, packed);
-        }
-        l += rs;
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&sm->p_full[s]);
-      }
-      if (!ok) break;
-      // epilogue: o = O / l, bf16, 16-byte stores of the valid rows
-      if (!mbar_wait_warp(&sm->pv_done[s], (pv_phase + n) & 1u, sm, p.status)) break;
-      pv_phase += n + 1;
-      tc_fence_after();
-      const float inv = 1.0f / l;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (static_cast<int64_t>(wi.bh) * p.q_rows + wi.q_row + row) * D;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
-        tmem_wait_ld();
-        if (row < wi.q_len) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
-            w.y = pack_bf16(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
-            w.z = pack_bf16(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
-            w.w = pack_bf16(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
-            dst[v] = w;
-          }
-        }
-      }
-      tc_fence_before();
-    }
+    // -------------------------------------------------------------- softmax warpgroups
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    softmax_role(sm, p, tmem, warp);
   }
 
   tc_fence_before();
@@ -554,32 +507,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// bf16 tensor [z][rows][128] as a 3-D map with 64 x 128 boxes and 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t zdim) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(zdim)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 }  // namespace

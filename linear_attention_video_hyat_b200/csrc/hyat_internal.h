@@ -64,8 +64,10 @@ struct SegStateArgs {
   int32_t nseg, seg_base, seg_stride, seg_len;
   float* out;                 // [BH][nseg][E], E = d*d + d (S row-major [a][b], then z[a])
   int32_t accumulate;         // out += instead of out =
+  uint32_t* status;           // device status word (tensor-core kernel's bounded waits)
 };
 cudaError_t launch_seg_state(const SegStateArgs& a, cudaStream_t s);
+cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t s);
 
 struct ComplementArgs {
   const float* sseg;          // [BH][nseg][E]

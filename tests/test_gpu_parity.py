@@ -133,8 +133,19 @@ def test_stream_small_steps_and_state():
     k_all, v_all = np.concatenate(kh, axis=2), np.concatenate(vh, axis=2)
     # after step 7 the state holds phi(k) v^T of every chunk evicted up to step 7
     S_ref, z_ref = oracle.stream_evicted_state(k_all, v_all, 7, w.chunk_tokens, 3)
-    np.testing.assert_allclose(S.reshape(1, 2, 128, 128), S_ref, rtol=0, atol=1e-5 * np.abs(S_ref).max())
-    np.testing.assert_allclose(z.reshape(1, 2, 128), z_ref, rtol=0, atol=1e-5 * np.abs(z_ref).max())
+    # The tensor-core fold takes phi(k) as a bf16 operand: each product phi(k)_a v_b carries a
+    # relative rounding error <= 2^-8 (v is exact), so |S - S*|_ab <= 2^-8 sum_j |phi(k_j)_a v_jb|;
+    # fp32 accumulation adds at most 1e-5 of the largest entry.
+    n_ev = (7 - 3 + 1) * w.chunk_tokens
+    pk = oracle.phi_elu1(k_all[:, :, :n_ev])
+    bound_S = 2.0 ** -8 * np.einsum("bhna,bhnc->bhac", pk, np.abs(v_all[:, :, :n_ev]))
+    bound_z = 2.0 ** -8 * pk.sum(axis=2)
+    err_S = np.abs(S.reshape(1, 2, 128, 128) - S_ref)
+    err_z = np.abs(z.reshape(1, 2, 128) - z_ref)
+    assert np.all(err_S <= bound_S + 1e-5 * np.abs(S_ref).max()), float((err_S / bound_S).max())
+    assert np.all(err_z <= bound_z + 1e-5 * np.abs(z_ref).max()), float((err_z / bound_z).max())
+    # and the error is the random rounding kind: its rms is far below the worst case
+    assert np.sqrt((err_S ** 2).mean()) < 0.1 * np.sqrt((bound_S ** 2).mean())
     h.close()
 
 
