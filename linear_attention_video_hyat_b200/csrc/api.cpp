@@ -21,7 +21,7 @@ enum Kind { K_STATE = 0, K_COMPLEMENT = 1, K_ATTN = 2, K_FOLD = 3, K_PREP = 4 };
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Plan {
-  size_t status = 0, work = 0, entries = 0, pairs = 0, cm = 0, sseg = 0, srest = 0, srest_t = 0;
+  size_t status = 0, work = 0, entries = 0, pairs = 0, cm = 0, sseg = 0, srest = 0, srest_bf16 = 0;
   size_t ring_k = 0, ring_v = 0, mask = 0, total = 0;
   int64_t n_work = 0, n_entries = 0;
 };
@@ -44,7 +44,7 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
   if (c.mode == HYAT_MODE_STREAM) {
     const int64_t Lc = stream_chunk_tokens(c), nwc = stream_window_chunks(c), nqt = tiles(Lc);
     p.srest = take(sizeof(float) * BH * E);
-    p.srest_t = take(2 * BH * c.d * c.d);
+    p.srest_bf16 = take(2 * BH * c.d * c.d);
     p.ring_k = take(size_t(BH * nwc * Lc * c.d * elem_bytes(c)));
     p.ring_v = take(size_t(BH * nwc * Lc * c.d * elem_bytes(c)));
     p.mask = take(size_t(c.mask_heads) * nqt * nqt * nwc);
@@ -52,7 +52,7 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
     p.cm = take(sizeof(float) * size_t(L.cm_heads) * L.nqg * L.nseg);
     p.sseg = take(sizeof(float) * BH * L.nseg * E);
     p.srest = take(sizeof(float) * BH * L.nqg * E);
-    p.srest_t = take(2 * BH * L.nqg * c.d * c.d);
+    p.srest_bf16 = take(2 * BH * L.nqg * c.d * c.d);
   }
   p.total = off;
   return p;
@@ -101,7 +101,7 @@ struct hyat_ctx {
   float* d_cm = nullptr;
   float* d_sseg = nullptr;
   float* d_srest = nullptr;
-  uint16_t* d_srest_t = nullptr;
+  uint16_t* d_srest_bf16 = nullptr;
   void* d_ring_k = nullptr;
   void* d_ring_v = nullptr;
   uint8_t* d_mask = nullptr;
@@ -173,7 +173,7 @@ AttnArgs attn_args(hyat_ctx* h, const void* q, const void* k, const void* v, voi
   a.pairs = h->d_pairs;
   a.n_pairs = h->n_pairs;
   a.srest = h->d_srest;
-  a.srest_t = h->d_srest_t;
+  a.srest_bf16 = h->d_srest_bf16;
   a.nqg = nqg;
   a.d = h->cfg.d;
   a.dtype = h->cfg.dtype;
@@ -185,16 +185,9 @@ AttnArgs attn_args(hyat_ctx* h, const void* q, const void* k, const void* v, voi
 }
 
 hyat_status launch_attention(hyat_ctx* h, const AttnArgs& a, cudaStream_t s) {
-  cudaError_t e;
-  if (h->use_tc) {
-    e = timed(h, K_PREP, s, [&] {
-      return launch_state_transpose_bf16(h->d_srest, h->d_srest_t, int64_t(h->BH) * a.nqg, h->cfg.d, s);
-    });
-    if (e != cudaSuccess) return cuda_fail(h, e, "state transpose");
-    e = timed(h, K_ATTN, s, [&] { return launch_attn_tc(a, h->num_sms, s); });
-  } else {
-    e = timed(h, K_ATTN, s, [&] { return launch_attn_simt(a, s); });
-  }
+  cudaError_t e = timed(h, K_ATTN, s, [&] {
+    return h->use_tc ? launch_attn_tc(a, h->num_sms, s) : launch_attn_simt(a, s);
+  });
   if (e != cudaSuccess) return cuda_fail(h, e, "attention kernel");
   return HYAT_OK;
 }
@@ -262,7 +255,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   h->d_entries = reinterpret_cast<Entry*>(ws + h->plan.entries);
   h->d_pairs = reinterpret_cast<int4*>(ws + h->plan.pairs);
   h->d_srest = reinterpret_cast<float*>(ws + h->plan.srest);
-  h->d_srest_t = reinterpret_cast<uint16_t*>(ws + h->plan.srest_t);
+  h->d_srest_bf16 = reinterpret_cast<uint16_t*>(ws + h->plan.srest_bf16);
   if (cfg->mode == HYAT_MODE_STREAM) {
     h->d_ring_k = ws + h->plan.ring_k;
     h->d_ring_v = ws + h->plan.ring_v;
@@ -340,7 +333,10 @@ hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const vo
   if (e != cudaSuccess) return cuda_fail(h, e, "segment state kernel");
   ComplementArgs ca{};
   ca.sseg = h->d_sseg; ca.cm = h->d_cm; ca.srest = h->d_srest;
+  ca.srest_bf16 = h->use_tc ? h->d_srest_bf16 : nullptr;
+  ca.write_f32_s = h->use_tc ? 0 : 1;       // the tensor-core path reads S as bf16, z as fp32
   ca.BH = h->BH; ca.H = h->cfg.H; ca.cm_heads = L.cm_heads; ca.nseg = L.nseg; ca.nqg = L.nqg; ca.E = h->E;
+  ca.d = h->cfg.d;
   e = timed(h, K_COMPLEMENT, s, [&] { return launch_complement(ca, s); });
   if (e != cudaSuccess) return cuda_fail(h, e, "complement kernel");
   return launch_attention(h, attn_args(h, q, k, v, o, h->plan.n_work, L.nqg), s);
@@ -383,6 +379,10 @@ hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, co
       sa.out = h->d_srest; sa.accumulate = 1; sa.status = h->d_status;
       cudaError_t e2 = h->use_tc ? launch_seg_state_tc(sa, h->num_sms, s) : launch_seg_state(sa, s);
       if (e2 != cudaSuccess) return e2;
+      if (h->use_tc) {
+        e2 = launch_state_to_bf16(h->d_srest, h->d_srest_bf16, h->BH, c.d, s);
+        if (e2 != cudaSuccess) return e2;
+      }
     }
     RingCopyArgs ra{};
     ra.k = k; ra.v = v; ra.ring_k = h->d_ring_k; ra.ring_v = h->d_ring_v;
@@ -510,6 +510,8 @@ hyat_status hyat_stream_set_state(hyat_handle h, const void* src_host, size_t by
   e = cudaMemcpy(h->d_srest, p, sb, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(h->d_ring_k, p + sb, rb, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(h->d_ring_v, p + sb + rb, rb, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && h->use_tc) e = launch_state_to_bf16(h->d_srest, h->d_srest_bf16, h->BH, h->cfg.d, nullptr);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(h, e, "state copy");
   h->step = hd.step;
   return HYAT_OK;

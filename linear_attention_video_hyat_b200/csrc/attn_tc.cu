@@ -13,15 +13,16 @@
 // Design for B200:
 //   * one persistent CTA per SM; a CTA owns a pair of 128-row query tiles
 //     ("slots"), so the softmax of one slot overlaps the MMAs of the other;
-//   * warp 8 issues TMA loads (Q tiles, K/V tiles, S_rest^T) into 128B-swizzled
+//   * warp 8 issues TMA loads (Q tiles, K/V tiles, bf16 S_rest) into 128B-swizzled
 //     shared memory through a 5-stage ring; warp 9 issues tcgen05.mma (one
 //     thread) with fp32 accumulators in TMEM; warps 0-3 / 4-7 run the softmax
 //     of slot 0 / 1, one query row per thread, reading S from TMEM and writing
 //     P (bf16) back into TMEM, where it is the A operand of the P.V MMA;
 //   * TMEM (512 columns): S0 | S1 | O0 | O1, each 128 columns; P and phi(Q)
 //     alias the first 64 columns of S;
-//   * the running max is only moved when it grows by more than 8 (log2
-//     units): the rescale of O in TMEM is rare and the result is exact;
+//   * no per-tile row max: exponents use the row's current reference m, and m
+//     moves (with a rescale of O in TMEM) only when the running sum would leave
+//     the safe fp32 range, which keeps the result exact and the rescale rare;
 //   * every mbarrier wait is bounded (%globaltimer); a wait that gives up sets
 //     the status word, and all roles drain and free TMEM before exiting.
 #include <cuda.h>
@@ -48,13 +49,9 @@ constexpr int MMA_WARP = 9;
 // and 1 warp of group 2 = 2 x 32 x 208 + 32 x 88 = 16128 <= 16384.
 constexpr int kRegsSoftmax = 208;
 constexpr int kRegsLoadMma = 88;
-constexpr float kRescaleThreshold = 8.0f;        // log2 units
-// Of every 8 score pairs of a full tile, this many take exp2 on the FMA pipe (exp2_fma) and
-// the rest on MUFU, so the two pipes share the exponentials; partial tiles use MUFU only.
-#ifndef HYAT_EMU_OF8
-#define HYAT_EMU_OF8 0
-#endif
-constexpr int kEmuOf8 = HYAT_EMU_OF8;
+// The reference max m of a row moves only when the running sum l would leave the safe fp32
+// range: every exponent uses the same m as its row's accumulators, so the result is exact.
+constexpr float kSafeSum = 1.2676506e30f;        // 2^100
 
 // instruction descriptor, kind::f16: D f32, A/B bf16, M = 128, N = 128
 constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -113,6 +110,26 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* b, uint32_t parity, Sme
 __device__ __forceinline__ bool wait_warp(uint64_t* b, uint32_t parity, Smem* sm, uint32_t* status) {
   if (__all_sync(0xffffffffu, mbar_try_wait(b, parity))) return true;
   return mbar_wait_warp(b, parity, sm, status);
+}
+
+// p = 2^(s * sl + neg_m) for the 128 scores of this row; P (bf16 pairs) -> TMEM at tS.
+// Returns the row sum of p (fp32, 8 partial sums).
+__device__ __forceinline__ float exp_tile(const uint32_t (&r)[128], float sl, float neg_m, uint32_t tS) {
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float p0 = ex2(fmaf(u2f(r[h * 64 + 2 * i]), sl, neg_m));
+      const float p1 = ex2(fmaf(u2f(r[h * 64 + 2 * i + 1]), sl, neg_m));
+      acc[(2 * i) & 7] += p0;
+      acc[(2 * i + 1) & 7] += p1;
+      pk[i] = pack_bf16(p0, p1);
+    }
+    tmem_st32(tS + h * 32, pk);
+  }
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
 // One query row per thread (TMEM lane = row). Slot s = warpgroup index.
@@ -184,21 +201,22 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
 #pragma unroll
         for (int i = 0; i < 128; ++i) r[i] = i < klen ? r[i] : 0xff800000u;   // -inf
       }
-      // row max: 8 independent chains of 3-input max, then a short tree
-      float mx[8];
+      // Optimistic pass: p = 2^(s * scale_log2 - m) with the row's current reference m.
+      float rs = exp_tile(r, sl, -m, tS);
+      // Rare slow path: the sum left the safe range (a score far above m). Move m to the row
+      // max, rescale O and l (after the previous P.V has landed), and redo the tile.
+      if (__any_sync(0xffffffffu, !(l + rs < kSafeSum))) {
+        float mx[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float a = fmax3(u2f(r[k]), u2f(r[k + 8]), u2f(r[k + 16]));
+        for (int k = 0; k < 8; ++k) {
+          float a = fmax3(u2f(r[k]), u2f(r[k + 8]), u2f(r[k + 16]));
 #pragma unroll
-        for (int t = 3; t < 15; t += 2) a = fmax3(a, u2f(r[k + 8 * t]), u2f(r[k + 8 * t + 8]));
-        mx[k] = fmaxf(a, u2f(r[k + 120]));
-      }
-      const float mrow = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
-      const float m_cand = mrow * sl;
-      if (__any_sync(0xffffffffu, m_cand > m + kRescaleThreshold)) {
-        const float m_new = fmaxf(m, m_cand);
+          for (int t = 3; t < 15; t += 2) a = fmax3(a, u2f(r[k + 8 * t]), u2f(r[k + 8 * t + 8]));
+          mx[k] = fmaxf(a, u2f(r[k + 120]));
+        }
+        const float mrow = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
+        const float m_new = fmaxf(m, mrow * sl);
         const float alpha = ex2(m - m_new);
-        // the previous P.V (or the linear-branch MMA) must be complete before O is rescaled
         if (!wait_warp(pv_done, (pv_phase + j) & 1u, sm, p.status)) return;
         tc_fence_after();
 #pragma unroll
@@ -213,42 +231,9 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
         tmem_wait_st();
         l *= alpha;
         m = m_new;
+        rs = exp_tile(r, sl, -m, tS);
       }
-      const float neg_m = -m;
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (kEmuOf8 > 0 && klen == 128) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x0 = fmaf(u2f(r[h * 64 + 2 * i]), sl, neg_m);
-            const float x1 = fmaf(u2f(r[h * 64 + 2 * i + 1]), sl, neg_m);
-            const bool emu = (i & 7) < kEmuOf8;
-            const float p0 = emu ? exp2_fma(x0) : ex2(x0);
-            const float p1 = emu ? exp2_fma(x1) : ex2(x1);
-            acc[(2 * i) & 7] += p0;
-            acc[(2 * i + 1) & 7] += p1;
-            pk[i] = pack_bf16(p0, p1);
-          }
-          tmem_st32(tS + h * 32, pk);
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2(fmaf(u2f(r[h * 64 + 2 * i]), sl, neg_m));
-            const float p1 = ex2(fmaf(u2f(r[h * 64 + 2 * i + 1]), sl, neg_m));
-            acc[(2 * i) & 7] += p0;
-            acc[(2 * i + 1) & 7] += p1;
-            pk[i] = pack_bf16(p0, p1);
-          }
-          tmem_st32(tS + h * 32, pk);
-        }
-      }
-      l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      l += rs;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -413,7 +398,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto linear = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
         const uint32_t sb = smem_u32(sm->kv[stage]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, desc_kmajor(sb, kk), kIdescKK, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, desc_mnmajor(sb, kk), kIdescKMN, kk > 0);
         mma_commit(done);
       };
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
@@ -423,7 +408,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int n0 = p.work[pr.x].entry_end - p.work[pr.x].entry_begin;
         const int n1 = has1 ? p.work[pr.y].entry_end - p.work[pr.y].entry_begin : 0;
         int k0 = -1, k1 = -1, v0 = -1, v1 = -1, sst = -1;
-        // slot 0: O0 = phi(Q0) S_rest^T, then S0 = Q0 K^T
+        // slot 0: O0 = phi(Q0) S_rest (S_rest [a][b] is the MN-major B operand), then S0 = Q0 K^T
         ok = wait_p(&sm->p_full[0], pph0) && next_stage(sst);
         if (!ok) break;
         linear(tO0, tS0, sst, &sm->pv_done[0]);
@@ -517,7 +502,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s) {
   if (a.n_pairs == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv, ms;
   if (!make_map(&mq, a.q, a.q_rows, a.BH) || !make_map(&mk, a.k, a.k_rows, a.BH) ||
-      !make_map(&mv, a.v, a.k_rows, a.BH) || !make_map(&ms, a.srest_t, D, int64_t(a.BH) * a.nqg))
+      !make_map(&mv, a.v, a.k_rows, a.BH) || !make_map(&ms, a.srest_bf16, D, int64_t(a.BH) * a.nqg))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {

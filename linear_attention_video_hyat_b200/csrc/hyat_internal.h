@@ -72,14 +72,17 @@ cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t
 struct ComplementArgs {
   const float* sseg;          // [BH][nseg][E]
   const float* cm;            // [cm_heads][nqg][nseg]
-  float* srest;               // [BH][nqg][E]
-  int32_t BH, H, cm_heads, nseg, nqg, E;
+  float* srest;               // [BH][nqg][E]: z always; S only if write_f32_s
+  uint16_t* srest_bf16;       // [BH][nqg][d][d] bf16 S (natural [a][b] layout) or null
+  int32_t write_f32_s;
+  int32_t BH, H, cm_heads, nseg, nqg, E, d;
 };
 cudaError_t launch_complement(const ComplementArgs& a, cudaStream_t s);
 
-// S (fp32 [a][b] then z) -> bf16 S^T [b][a] for the tensor-core linear term.
-cudaError_t launch_state_transpose_bf16(const float* srest, uint16_t* st, int64_t n_groups,
-                                        int32_t d, cudaStream_t s);
+// S (fp32 [a][b], group stride d*d + d) -> bf16 S [a][b] (group stride d*d) for the
+// tensor-core linear term, where S in its natural layout is the MN-major B operand.
+cudaError_t launch_state_to_bf16(const float* srest, uint16_t* out, int64_t n_groups, int32_t d,
+                                 cudaStream_t s);
 
 struct AttnArgs {
   const void* q; const void* k; const void* v; void* o;
@@ -88,7 +91,7 @@ struct AttnArgs {
   const Entry* entries;
   const int4* pairs; int32_t n_pairs;   // tensor-core path: {item0, item1 or -1, shared list, 0}
   const float* srest;         // [BH][nqg][E]
-  const uint16_t* srest_t;    // [BH][nqg][d][d] bf16 (tensor-core path)
+  const uint16_t* srest_bf16; // [BH][nqg][d][d] bf16 S, natural layout (tensor-core path)
   int32_t nqg, d, dtype, BH;
   float scale_log2;           // scale * log2(e)
   uint32_t* status;

@@ -134,25 +134,28 @@ __global__ void __launch_bounds__(256) complement_kernel(ComplementArgs a) {
     }
   }
   if (e < a.E) {
+    const int64_t dd = static_cast<int64_t>(a.d) * a.d;
+    const bool is_s = e < dd;
 #pragma unroll
-    for (int gg = 0; gg < 32; ++gg)
-      if (g0 + gg < a.nqg) a.srest[(static_cast<int64_t>(bh) * a.nqg + g0 + gg) * a.E + e] = acc[gg];
+    for (int gg = 0; gg < 32; ++gg) {
+      if (g0 + gg >= a.nqg) continue;
+      const int64_t grp = static_cast<int64_t>(bh) * a.nqg + g0 + gg;
+      if (!is_s || a.write_f32_s) a.srest[grp * a.E + e] = acc[gg];
+      if (is_s && a.srest_bf16) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(acc[gg]);
+        a.srest_bf16[grp * dd + e] = *reinterpret_cast<const uint16_t*>(&h);
+      }
+    }
   }
 }
 
-// S [a][b] fp32 (row stride d, group stride d*d + d) -> S^T [b][a] bf16 (group stride d*d)
-__global__ void state_transpose_kernel(const float* __restrict__ s, uint16_t* __restrict__ st,
-                                       int32_t d) {
-  __shared__ float tile[32][33];
-  const int64_t g = blockIdx.z;
-  const int a0 = blockIdx.y * 32, b0 = blockIdx.x * 32;
-  const float* S = s + g * (static_cast<int64_t>(d) * d + d);
-  uint16_t* T = st + g * static_cast<int64_t>(d) * d;
-  for (int r = threadIdx.y; r < 32; r += 8) tile[r][threadIdx.x] = S[static_cast<int64_t>(a0 + r) * d + b0 + threadIdx.x];
-  __syncthreads();
-  for (int r = threadIdx.y; r < 32; r += 8) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(tile[threadIdx.x][r]);
-    T[static_cast<int64_t>(b0 + r) * d + a0 + threadIdx.x] = *reinterpret_cast<const uint16_t*>(&h);
+// S [a][b] fp32 (group stride d*d + d) -> bf16 S [a][b] (group stride d*d)
+__global__ void state_to_bf16_kernel(const float* __restrict__ s, uint16_t* __restrict__ out, int64_t n, int32_t d) {
+  const int64_t dd = static_cast<int64_t>(d) * d;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n; i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t g = i / dd, e = i % dd;
+    const __nv_bfloat16 h = __float2bfloat16_rn(s[g * (dd + d) + e]);
+    out[i] = *reinterpret_cast<const uint16_t*>(&h);
   }
 }
 
@@ -414,11 +417,11 @@ cudaError_t launch_complement(const ComplementArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_state_transpose_bf16(const float* srest, uint16_t* st, int64_t n_groups, int32_t d,
-                                        cudaStream_t s) {
-  if (n_groups == 0) return cudaSuccess;
-  dim3 grid(d / 32, d / 32, static_cast<unsigned>(n_groups));
-  state_transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(srest, st, d);
+cudaError_t launch_state_to_bf16(const float* srest, uint16_t* out, int64_t n_groups, int32_t d, cudaStream_t s) {
+  const int64_t n = n_groups * d * d;
+  if (n == 0) return cudaSuccess;
+  const int blocks = static_cast<int>((n + 255) / 256 < 2048 ? (n + 255) / 256 : 2048);
+  state_to_bf16_kernel<<<blocks, 256, 0, s>>>(srest, out, n, d);
   return cudaGetLastError();
 }
 

@@ -85,7 +85,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   const size_t o_cm = take(sizeof(float) * L.cm.size());
   const size_t o_sseg = take(sizeof(float) * size_t(BH) * L.nseg * E);
   const size_t o_srest = take(sizeof(float) * size_t(BH) * L.nqg * E);
-  const size_t o_srest_t = take(2 * size_t(BH) * L.nqg * cfg->d * cfg->d);
+  const size_t o_srest_bf16 = take(2 * size_t(BH) * L.nqg * cfg->d * cfg->d);
   if (off > kNoAllocScratchBytes) return HYAT_ERR_UNSUPPORTED;  // needs more than the static scratch
 
   void* base = nullptr;
@@ -118,6 +118,15 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   ca.srest = reinterpret_cast<float*>(ws + o_srest);
   ca.BH = static_cast<int32_t>(BH); ca.H = cfg->H; ca.cm_heads = L.cm_heads; ca.nseg = L.nseg; ca.nqg = L.nqg;
   ca.E = static_cast<int32_t>(E);
+  ca.d = cfg->d;
+  int major = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return HYAT_ERR_CUDA;
+  const bool use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
+                      attn_tc_supported(cfg->d, cfg->dtype);
+  ca.srest_bf16 = use_tc ? reinterpret_cast<uint16_t*>(ws + o_srest_bf16) : nullptr;
+  ca.write_f32_s = use_tc ? 0 : 1;
   if (launch_complement(ca, s) != cudaSuccess) return HYAT_ERR_CUDA;
 
   AttnArgs a{};
@@ -129,22 +138,13 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   a.pairs = reinterpret_cast<const int4*>(ws + o_pairs);
   a.n_pairs = static_cast<int32_t>(pairs.size());
   a.srest = ca.srest;
-  a.srest_t = reinterpret_cast<const uint16_t*>(ws + o_srest_t);
+  a.srest_bf16 = reinterpret_cast<const uint16_t*>(ws + o_srest_bf16);
   a.nqg = L.nqg; a.d = cfg->d; a.dtype = cfg->dtype; a.BH = static_cast<int32_t>(BH);
   const float scale = cfg->scale > 0.0f ? cfg->scale : 1.0f / sqrtf(float(cfg->d));
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = reinterpret_cast<uint32_t*>(ws + o_status);
 
-  int major = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-    return HYAT_ERR_CUDA;
-  const bool use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
-                      attn_tc_supported(cfg->d, cfg->dtype);
   if (use_tc) {
-    if (launch_state_transpose_bf16(ca.srest, reinterpret_cast<uint16_t*>(ws + o_srest_t), BH * L.nqg, cfg->d, s) !=
-        cudaSuccess)
-      return HYAT_ERR_CUDA;
     if (launch_attn_tc(a, num_sms, s) != cudaSuccess) return HYAT_ERR_CUDA;
   } else {
     if (launch_attn_simt(a, s) != cudaSuccess) return HYAT_ERR_CUDA;

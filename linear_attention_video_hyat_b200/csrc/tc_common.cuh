@@ -149,21 +149,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
-// 2^x on the FMA pipe, for x <= 8: Cody-Waite range reduction x = n + f with n = round(x)
-// (the 1.5 * 2^23 shifter leaves n in the low mantissa bits of t) and f in [-1/2, 1/2], a
-// degree-3 polynomial for 2^f (coefficients fitted for minimax relative error on [-1/2, 1/2];
-// max relative error 7.5e-5, below the 2^-9 half-ulp of the bf16 operand it feeds), and the
-// scale 2^n added into the exponent field. Inputs below -126 clamp to about 2^-126.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  const float p = fmaf(fmaf(fmaf(0.05517605319619179f, f, 0.24261149764060974f), f, 0.6932601928710938f), f,
-                       0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

@@ -52,6 +52,18 @@ def test_window_small(dtype, T, F, C, h, d, H):
     assert_parity(dtype, f64(o), _window_ref(w, q, k, v), (T, F, C, h, d, H))
 
 
+@pytest.mark.parametrize("sigma", [6.0, 20.0])
+def test_window_large_logits(sigma):
+    """Scores far above the reference max (sigma 20: |s| * log2(e) / sqrt(d) reaches ~250):
+    the kernel must move its reference max and rescale the accumulator exactly."""
+    w = wl.Workload("large_logits", "window", 1, 2, 128, 300, 4, 2, 1, seed=17)
+    q, k, v = wl.gen_qkv(w)
+    q = (q.float() * sigma).to(torch.bfloat16)
+    k = (k.float() * sigma).to(torch.bfloat16)
+    o, _ = _bidir(w, qkv=(q, k, v))
+    assert_parity("bf16", f64(o), _window_ref(w, q, k, v), sigma)
+
+
 def test_window_batch2_per_head_std():
     w = wl.Workload("small_b2", "window", 2, 3, 128, 250, 6, 3, 1, per_head_std=True, seed=11)
     o, (q, k, v) = _bidir(w)
