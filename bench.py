@@ -240,8 +240,8 @@ def main():
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
 
-    h.set_profiling(True)
-    h.kernel_times()
+    # Pass 1 (the headline): K steps, no per-launch events, so the kernels of a step overlap
+    # their launches (programmatic dependent launch) exactly as in production.
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         t0.record(stream)
@@ -251,13 +251,21 @@ def main():
         torch.cuda.synchronize(dev)
     h.sync()
     ms = t0.elapsed_time(t1) / a.steps
+    # Pass 2: K more steps with CUDA events around every launch (library-side), for the
+    # per-kernel durations of the roofline.
+    h.set_profiling(True)
+    h.kernel_times()
+    with ClockSampler(local) as clk2:
+        for _ in range(a.steps):
+            h.forward(qd, kd, vd, out=od)
+        torch.cuda.synchronize(dev)
     kt = h.kernel_times()
     h.set_profiling(False)
     if world > 1:
         mt = torch.tensor([ms], device=dev)
         torch.distributed.all_reduce(mt, op=torch.distributed.ReduceOp.MAX)
         ms = float(mt.item())
-    launches = sum(n for _, n in kt.values())
+    launches = sum(n for _, n in kt.values())   # per-step launches x K (pass 2 mirrors pass 1)
 
     value = counts["total_flops"] * world / (ms / 1e3) / 1e12
     tokens_per_s = w.B * w.N * world / (ms / 1e3)
@@ -272,6 +280,8 @@ def main():
         if t.get("source_sha256") == sha and t.get("workload") == w.name:
             traffic = t.get("dram_bytes_per_launch")
     roofline = {"bound": "tensor", "kernel": "attention", "achieved": achieved,
+                "timing": "per-launch CUDA events over a second pass of the same K steps",
+                "clocks_kernel_pass": clk2.summary(),
                 "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                 "peak_kind": f"{pk_src} bf16 burst", "peak_sustained": pk["bf16_tflops_sustained"],
                 "frac_sustained": achieved / pk["bf16_tflops_sustained"], "traffic": traffic,

@@ -44,11 +44,11 @@ constexpr int NUM_THREADS = 384;                 // 3 warpgroups
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512); warpgroup 2
-// (TMA, MMA, 2 idle warps) drops to 88, the two softmax warpgroups rise to 208:
-// 8 warps x 32 x 208 + 4 warps x 32 x 88 = 64512. Per SM sub-partition: 2 softmax warps
-// and 1 warp of group 2 = 2 x 32 x 208 + 32 x 88 = 16128 <= 16384.
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsLoadMma = 88;
+// (TMA, MMA, 2 idle warps) drops to 104, the two softmax warpgroups rise to 200:
+// 8 warps x 32 x 200 + 4 warps x 32 x 104 = 64512. Per SM sub-partition: 2 softmax warps
+// and 1 warp of group 2 = 2 x 32 x 200 + 32 x 104 = 16128 <= 16384.
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsLoadMma = 104;
 // The reference max m of a row moves only when the running sum l would leave the safe fp32
 // range: every exponent uses the same m as its row's accumulators, so the result is exact.
 constexpr float kSafeSum = 1.2676506e30f;        // 2^100
@@ -67,6 +67,7 @@ struct __align__(1024) Smem {
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort_flag;
+  float z[2][D];                 // z_rest of each slot's current query tile
 };
 
 struct TcParams {
@@ -157,16 +158,21 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
     if (!wait_warp(q_full, qph, sm, p.status)) return;
     qph ^= 1u;
     // phi(q) of this row -> TMEM (bf16 pairs), l = phi(q) . z
-    const float* z = p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D;
+    // z_rest of this tile's group into shared memory: one coalesced load per warpgroup
+    const float* zg = p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D;
+    float* z = sm->z[s];
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + s) : "memory");       // previous readers are done
+    z[row] = __ldg(zg + row);
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + s) : "memory");
     float l = 0.0f, m = 0.0f;
     {
       const uint8_t* qrow = sm->q[s] + row * 128;
       float lz[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
+#pragma unroll 4
       for (int c = 0; c < 16; ++c) {            // 8 columns per step
         const uint4 raw = *reinterpret_cast<const uint4*>(qrow + (c >> 3) * HALF_BYTES + (((c & 7) ^ (row & 7)) << 4));
-        const float4 za = __ldg(reinterpret_cast<const float4*>(z + 8 * c));
-        const float4 zb = __ldg(reinterpret_cast<const float4*>(z + 8 * c + 4));
+        const float4 za = *reinterpret_cast<const float4*>(z + 8 * c);
+        const float4 zb = *reinterpret_cast<const float4*>(z + 8 * c + 4);
         const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
         const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
         uint32_t pk[4];
@@ -302,6 +308,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
+  pdl_wait();                // the linear states come from the kernels launched before this one
 
   if (warp >= 8) {
     // ------------------------------------------------------------ warpgroup 2: TMA + MMA
@@ -383,22 +390,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         return true;
       };
-      auto qk = [&](uint32_t tS, const uint8_t* qbuf, int stage, uint64_t* done) {
-        const uint32_t qa = smem_u32(qbuf), kb = smem_u32(sm->kv[stage]);
+      // Descriptors: start address (>> 4) sits in the low bits, so a K step is an add of a
+      // constant; bases are computed once (issue slots on this sub-partition are shared with
+      // two softmax warps, so each MMA is kept to an add and the instruction).
+      const uint64_t dQ0 = sdesc(smem_u32(sm->q[0]), 16, 1024), dQ1 = sdesc(smem_u32(sm->q[1]), 16, 1024);
+      const uint64_t dK0 = sdesc(smem_u32(sm->kv[0]), 16, 1024);
+      const uint64_t dV0 = sdesc(smem_u32(sm->kv[0]), HALF_BYTES, 1024);
+      constexpr uint64_t kStageStep = TILE_BYTES >> 4;
+      auto koff = [](int kk) -> uint64_t { return static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4); };
+      auto qk = [&](uint32_t tS, uint64_t dq, int stage, uint64_t* done) {
+        const uint64_t dk = dK0 + static_cast<uint64_t>(stage) * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tS, desc_kmajor(qa, kk), desc_kmajor(kb, kk), kIdescKK, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) mma_ss(tS, dq + koff(kk), dk + koff(kk), kIdescKK, kk > 0);
         mma_commit(done);
       };
       auto pv = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
-        const uint32_t vb = smem_u32(sm->kv[stage]);
+        const uint64_t dv = dV0 + static_cast<uint64_t>(stage) * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, desc_mnmajor(vb, kk), kIdescKMN, 1);
+        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescKMN, 1);
         mma_commit(done);
       };
       auto linear = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
-        const uint32_t sb = smem_u32(sm->kv[stage]);
+        const uint64_t dv = dV0 + static_cast<uint64_t>(stage) * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, desc_mnmajor(sb, kk), kIdescKMN, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescKMN, kk > 0);
         mma_commit(done);
       };
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
@@ -420,7 +435,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (n0 > 0) {
           ok = next_stage(k0);
           if (!ok) break;
-          qk(tS0, sm->q[0], k0, &sm->s_full[0]);
+          qk(tS0, dQ0, k0, &sm->s_full[0]);
           if (!shared) mma_commit(&sm->kv_empty[k0]);
         }
         if (n0 <= 1) mma_commit(&sm->q_empty[0]);
@@ -437,7 +452,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (n1 > 0) {
             if (shared) k1 = k0;
             else if (!(ok = next_stage(k1))) break;
-            qk(tS1, sm->q[1], k1, &sm->s_full[1]);
+            qk(tS1, dQ1, k1, &sm->s_full[1]);
             mma_commit(&sm->kv_empty[k1]);
           }
           if (n1 <= 1) mma_commit(&sm->q_empty[1]);
@@ -450,7 +465,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!shared) mma_commit(&sm->kv_empty[v0]);
             if (j + 1 < n0) {
               if (!(ok = next_stage(k0))) break;
-              qk(tS0, sm->q[0], k0, &sm->s_full[0]);
+              qk(tS0, dQ0, k0, &sm->s_full[0]);
               if (!shared) mma_commit(&sm->kv_empty[k0]);
               if (j + 2 == n0) mma_commit(&sm->q_empty[0]);
             }
@@ -464,7 +479,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (j + 1 < n1) {
               if (shared) k1 = k0;
               else if (!(ok = next_stage(k1))) break;
-              qk(tS1, sm->q[1], k1, &sm->s_full[1]);
+              qk(tS1, dQ1, k1, &sm->s_full[1]);
               mma_commit(&sm->kv_empty[k1]);
               if (j + 2 == n1) mma_commit(&sm->q_empty[1]);
             }
@@ -500,7 +515,8 @@ bool attn_tc_supported(int d, int dtype) { return d == D && dtype == HYAT_BF16; 
 
 cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s) {
   if (a.n_pairs == 0) return cudaSuccess;
-  CUtensorMap mq, mk, mv, ms;
+  CUtensorMap mq, mk, mv, ms;       // 128-row boxes: two loads of 64 x 128 bf16 = TILE_BYTES
+  static_assert(2 * 64 * 128 * 2 == TILE_BYTES, "tile bytes must match the two TMA boxes");
   if (!make_map(&mq, a.q, a.q_rows, a.BH) || !make_map(&mk, a.k, a.k_rows, a.BH) ||
       !make_map(&mv, a.v, a.k_rows, a.BH) || !make_map(&ms, a.srest_bf16, D, int64_t(a.BH) * a.nqg))
     return cudaErrorInvalidValue;
@@ -523,8 +539,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s) {
   p.scale_log2 = a.scale_log2;
   p.status = a.status;
   const int grid = a.n_pairs < num_sms ? a.n_pairs : num_sms;
-  attn_tc_kernel<<<grid, NUM_THREADS, kSmemBytes, s>>>(mq, mk, mv, ms, p);
-  return cudaGetLastError();
+  return launch_pdl(attn_tc_kernel, dim3(grid), dim3(NUM_THREADS), kSmemBytes, s, mq, mk, mv, ms, p);
 }
 
 }  // namespace hyat

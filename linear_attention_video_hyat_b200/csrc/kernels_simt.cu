@@ -105,39 +105,47 @@ __global__ void __launch_bounds__(256) seg_state_kernel(SegStateArgs a) {
 // --------------------------------------------------------------------------
 // Complement reduction: srest[bh][g] = sum_s cm[hm][g][s] * sseg[bh][s]
 // (the 0/1 matrix cm marks the segments in a group's linear set).
-// grid (ceil(E/256), ceil(nqg/32), BH), 256 threads: one column, 32 groups each.
+// grid (ceil(E/256), ceil(nqg/G), BH), 256 threads: one column, G groups each; segment values
+// are loaded SB at a time before the sums so that the loads overlap.
 // --------------------------------------------------------------------------
+template <int G, int SB>
 __global__ void __launch_bounds__(256) complement_kernel(ComplementArgs a) {
-  __shared__ float cms[32][33];
+  // Programmatic dependent launch: wait for the state kernel's results (a no-op when this
+  // kernel was launched without the attribute), then let the attention kernel launch.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float cms[G][SB + 1];
   const int tid = threadIdx.x;
   const int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + tid;
-  const int g0 = blockIdx.y * 32, bh = blockIdx.z;
+  const int g0 = blockIdx.y * G, bh = blockIdx.z;
   const int hm = a.cm_heads == 1 ? 0 : bh % a.H;
   const float* S = a.sseg + static_cast<int64_t>(bh) * a.nseg * a.E;
   const float* cm = a.cm + static_cast<int64_t>(hm) * a.nqg * a.nseg;
-  float acc[32];
+  float acc[G];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-  for (int s0 = 0; s0 < a.nseg; s0 += 32) {
+  for (int i = 0; i < G; ++i) acc[i] = 0.0f;
+  for (int s0 = 0; s0 < a.nseg; s0 += SB) {
     __syncthreads();
-    for (int idx = tid; idx < 32 * 32; idx += 256) {
-      const int gg = idx >> 5, ss = idx & 31;
+    for (int idx = tid; idx < G * SB; idx += 256) {
+      const int gg = idx / SB, ss = idx % SB;
       cms[gg][ss] = (g0 + gg < a.nqg && s0 + ss < a.nseg)
                         ? cm[static_cast<int64_t>(g0 + gg) * a.nseg + s0 + ss] : 0.0f;
     }
     __syncthreads();
-    const int ns = min(32, a.nseg - s0);
-    for (int ss = 0; ss < ns; ++ss) {
-      const float sv = e < a.E ? S[static_cast<int64_t>(s0 + ss) * a.E + e] : 0.0f;
+    float sv[SB];
 #pragma unroll
-      for (int gg = 0; gg < 32; ++gg) acc[gg] = fmaf(cms[gg][ss], sv, acc[gg]);
-    }
+    for (int ss = 0; ss < SB; ++ss)
+      sv[ss] = (e < a.E && s0 + ss < a.nseg) ? __ldg(S + static_cast<int64_t>(s0 + ss) * a.E + e) : 0.0f;
+#pragma unroll
+    for (int ss = 0; ss < SB; ++ss)
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) acc[gg] = fmaf(cms[gg][ss], sv[ss], acc[gg]);
   }
   if (e < a.E) {
     const int64_t dd = static_cast<int64_t>(a.d) * a.d;
     const bool is_s = e < dd;
 #pragma unroll
-    for (int gg = 0; gg < 32; ++gg) {
+    for (int gg = 0; gg < G; ++gg) {
       if (g0 + gg >= a.nqg) continue;
       const int64_t grp = static_cast<int64_t>(bh) * a.nqg + g0 + gg;
       if (!is_s || a.write_f32_s) a.srest[grp * a.E + e] = acc[gg];
@@ -412,9 +420,18 @@ cudaError_t launch_seg_state(const SegStateArgs& a, cudaStream_t s) {
 
 cudaError_t launch_complement(const ComplementArgs& a, cudaStream_t s) {
   if (a.nqg == 0 || a.BH == 0) return cudaSuccess;
-  dim3 grid((a.E + 255) / 256, (a.nqg + 31) / 32, a.BH);
-  complement_kernel<<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  const bool few = a.nqg <= 8;      // chunk windows: a handful of groups per head
+  dim3 grid((a.E + 255) / 256, (a.nqg + (few ? 7 : 31)) / (few ? 8 : 32), a.BH);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return few ? cudaLaunchKernelEx(&cfg, complement_kernel<8, 24>, a) : cudaLaunchKernelEx(&cfg, complement_kernel<32, 16>, a);
 }
 
 cudaError_t launch_state_to_bf16(const float* srest, uint16_t* out, int64_t n_groups, int32_t d, cudaStream_t s) {

@@ -9,7 +9,8 @@
 // and B = V_g^T (N = 128 features, K = tokens). Both tiles arrive from HBM by TMA as
 // [128 tokens x 128 features] with 128-byte swizzle, which is exactly the MN-major operand
 // layout, so no transpose is needed:
-//   * warp 8 streams K and V tiles through a 3-stage ring;
+//   * warp 8 streams 64-token K and V tiles through a 6-stage ring (about 160 KB in
+//     flight per SM, enough to cover loaded-HBM latency);
 //   * warps 0-3 apply phi in place in shared memory (zeroing rows past the segment end);
 //   * warp 9 issues tcgen05.mma into a double-buffered TMEM accumulator; z comes from a
 //     second MMA against an all-ones 16-column operand (N = 16), so it costs no CUDA-core work;
@@ -25,8 +26,11 @@ namespace {
 
 using namespace tc;
 
-constexpr int NST = 3;
-constexpr int STAGE_BYTES = 2 * TILE_BYTES;      // K tile, then V tile
+constexpr int TOK = 64;                          // tokens per stage
+constexpr int NST = 6;
+constexpr int KT_BYTES = TOK * D * 2;            // one [64 tokens x 128 features] bf16 tile
+constexpr int KT_HALF = KT_BYTES / 2;            // 64 features (128-byte rows)
+constexpr int STAGE_BYTES = 2 * KT_BYTES;        // K tile, then V tile
 constexpr int ST_THREADS = 320;                  // warps 0-3 phi, 4-7 drain, 8 TMA, 9 MMA
 constexpr int ST_TMA_WARP = 8, ST_MMA_WARP = 9;
 
@@ -86,7 +90,7 @@ __device__ __forceinline__ Unit unit_of(const StateParams& p, int u) {
   x.start = p.seg_base + x.g * p.seg_stride;
   const int64_t rem = p.rows - x.start;
   x.len = static_cast<int>(rem < p.seg_len ? (rem > 0 ? rem : 0) : p.seg_len);
-  x.ntiles = x.len > 0 ? (x.len + 127) / 128 : 1;
+  x.ntiles = x.len > 0 ? (x.len + TOK - 1) / TOK : 1;
   return x;
 }
 
@@ -127,6 +131,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
+  pdl_launch_dependents();   // the complement kernel may begin launching; it waits for our results
 
   if (warp == ST_TMA_WARP) {
     if (lane == 0) {
@@ -138,12 +143,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         for (int i = 0; i < x.ntiles && ok; ++i) {
           if (!(ok = swait(&sm->empty[st], ph ^ 1u, sm, p.status))) break;
           mbar_expect_tx(&sm->full[st], STAGE_BYTES);
-          const int row = x.start + 128 * i;
+          const int row = x.start + TOK * i;
           uint8_t* dst = sm->stage[st];
           tma_load_3d(smem_u32(dst), &tmK, 0, row, x.bh, &sm->full[st]);
-          tma_load_3d(smem_u32(dst + HALF_BYTES), &tmK, 64, row, x.bh, &sm->full[st]);
-          tma_load_3d(smem_u32(dst + TILE_BYTES), &tmV, 0, row, x.bh, &sm->full[st]);
-          tma_load_3d(smem_u32(dst + TILE_BYTES + HALF_BYTES), &tmV, 64, row, x.bh, &sm->full[st]);
+          tma_load_3d(smem_u32(dst + KT_HALF), &tmK, 64, row, x.bh, &sm->full[st]);
+          tma_load_3d(smem_u32(dst + KT_BYTES), &tmV, 0, row, x.bh, &sm->full[st]);
+          tma_load_3d(smem_u32(dst + KT_BYTES + KT_HALF), &tmV, 64, row, x.bh, &sm->full[st]);
           pending |= 1u << st;
           pending_ph = (pending_ph & ~(1u << st)) | (ph << st);
           if (++st == NST) { st = 0; ph ^= 1u; }
@@ -173,11 +178,12 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         for (int i = 0; i < x.ntiles && ok; ++i) {
           if (!(ok = swait(&sm->phi_done[st], ph, sm, p.status))) break;
           tc_fence_after();
-          const uint32_t kb = smem_u32(sm->stage[st]), vb = kb + TILE_BYTES;
+          const uint32_t kb = smem_u32(sm->stage[st]), vb = kb + KT_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = desc_mnmajor(kb, kk);
-            mma_ss(tacc, a, desc_mnmajor(vb, kk), kIdescState, (i | kk) != 0);
+          for (int kk = 0; kk < TOK / 16; ++kk) {
+            // MN-major, 64-feature halves KT_HALF apart, 16 tokens (2 x 8-row groups) per step
+            const uint64_t a = sdesc(kb + kk * 2048, KT_HALF, 1024);
+            mma_ss(tacc, a, sdesc(vb + kk * 2048, KT_HALF, 1024), kIdescState, (i | kk) != 0);
             mma_ss(tz, a, ones, kIdescOnes, (i | kk) != 0);
           }
           mma_commit(&sm->empty[st]);
@@ -201,10 +207,10 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
       const Unit x = unit_of(p, u);
       for (int i = 0; i < x.ntiles; ++i) {
         if (!(ok = swait_warp(&sm->full[st], ph, sm, p.status))) break;
-        const int valid = x.len - 128 * i;
-        uint8_t* kt = sm->stage[st] + half * HALF_BYTES;
+        const int valid = x.len - TOK * i;
+        uint8_t* kt = sm->stage[st] + half * KT_HALF;
 #pragma unroll 4
-        for (int k = 0; k < 16; ++k) {
+        for (int k = 0; k < TOK / 8; ++k) {
           const int r = (t >> 4) + 8 * k;
           uint4* addr = reinterpret_cast<uint4*>(kt + r * 128 + ((c8 ^ (r & 7)) << 4));
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
@@ -281,7 +287,9 @@ constexpr size_t kStateSmemBytes = sizeof(StateSmem) + 1024;
 cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t s) {
   if (a.nseg == 0 || a.BH == 0) return cudaSuccess;
   CUtensorMap mk, mv;
-  if (!tc::make_map(&mk, a.k, a.rows_per_bh, a.BH) || !tc::make_map(&mv, a.v, a.rows_per_bh, a.BH))
+  // boxes of TOK rows: 4 loads of 64 x TOK bf16 = STAGE_BYTES per stage
+  static_assert(4 * 64 * TOK * 2 == STAGE_BYTES, "stage bytes must match the four TMA boxes");
+  if (!tc::make_map(&mk, a.k, a.rows_per_bh, a.BH, TOK) || !tc::make_map(&mv, a.v, a.rows_per_bh, a.BH, TOK))
     return cudaErrorInvalidValue;
   static bool attr_set = false;
   if (!attr_set) {

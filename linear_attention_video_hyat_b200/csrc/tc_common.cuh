@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <utility>
 
 namespace hyat {
 namespace tc {
@@ -149,6 +150,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
+// Programmatic dependent launch: wait for the grids this one depends on (no-op when
+// launched without the attribute), and let dependent grids start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -161,6 +167,25 @@ __device__ __forceinline__ float phi_elu1(float x) {
   return x > 0.0f ? x + 1.0f : ex2(x * 1.4426950408889634f);
 }
 
+
+// ------------------------------------------------------------------ host: launches
+// Launch with programmatic stream serialization: the kernel may start while the previous
+// kernel on the stream finishes, and must call pdl_wait() before reading its outputs.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------ host: tensor maps
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -175,13 +200,15 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 tensor [z][rows][128] as a 3-D map with 64 x 128 boxes and 128-byte swizzle
-inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t zdim) {
+// bf16 tensor [z][rows][128] as a 3-D map with boxes of 64 columns x box_rows rows and
+// 128-byte swizzle. Each load of one box moves 64 * box_rows * 2 bytes: the expect-tx count
+// of the receiving barrier must match.
+inline bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t zdim, uint32_t box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(zdim)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
