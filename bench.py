@@ -77,6 +77,22 @@ def work_counts(w):
             "state_kernel_bytes": 2 * BH * N * d * 2 + BH * (N // w.tokens_per_frame) * (d * d + d) * 4}
 
 
+# ----------------------------------------------------------------- multi-rank
+def max_over_ranks(ms, device):
+    """The slowest rank's time (every rank calls this; identity on one process)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank, tokens_per_rank, ms_max, world):
+    """Whole-job effective TFLOP/s and tokens/s: every rank's units over the slowest rank's time."""
+    return flops_per_rank * world / (ms_max / 1e3) / 1e12, tokens_per_rank * world / (ms_max / 1e3)
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while the GPU runs."""
@@ -261,14 +277,10 @@ def main():
         torch.cuda.synchronize(dev)
     kt = h.kernel_times()
     h.set_profiling(False)
-    if world > 1:
-        mt = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(mt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(mt.item())
+    ms = max_over_ranks(ms, dev)
     launches = sum(n for _, n in kt.values())   # per-step launches x K (pass 2 mirrors pass 1)
 
-    value = counts["total_flops"] * world / (ms / 1e3) / 1e12
-    tokens_per_s = w.B * w.N * world / (ms / 1e3)
+    value, tokens_per_s = job_throughput(counts["total_flops"], w.B * w.N, ms, world)
     pk, pk_src = peaks()
     attn_ms = kt["attention"][0] / max(kt["attention"][1], 1)
     achieved = counts["attn_kernel_flops"] / (attn_ms / 1e3) / 1e12
@@ -311,13 +323,9 @@ def main():
             oh.copy_(od, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ems = e0.elapsed_time(e1) / e_steps
-        if world > 1:
-            mt = torch.tensor([ems], device=dev)
-            torch.distributed.all_reduce(mt, op=torch.distributed.ReduceOp.MAX)
-            ems = float(mt.item())
-        e2e = {"value": counts["total_flops"] * world / (ems / 1e3) / 1e12, "unit": "TFLOP/s",
-               "ms_per_step": ems, "tokens_per_s": w.B * w.N * world / (ems / 1e3),
+        ems = max_over_ranks(e0.elapsed_time(e1) / e_steps, dev)
+        e_value, e_tokens = job_throughput(counts["total_flops"], w.B * w.N, ems, world)
+        e2e = {"value": e_value, "unit": "TFLOP/s", "ms_per_step": ems, "tokens_per_s": e_tokens,
                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                "d2h_bytes_per_step": q.numel() * q.element_size()}
 

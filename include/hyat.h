@@ -86,6 +86,11 @@ typedef enum {
 
 /* Flags (hyat_config.flags). */
 #define HYAT_FLAG_SIMT 1u        /* run bf16 through the CUDA-core path (cross-check) */
+/* Test hook for the device-timeout path, which must work without faulting a GPU: the
+ * tensor-core attention kernel also waits once on a barrier that nothing signals, with a
+ * 20 ms limit. The wait gives up, every role drains and frees TMEM, the status word is set,
+ * and hyat_sync() returns HYAT_ERR_DEVICE_TIMEOUT; later calls on any handle work. */
+#define HYAT_FLAG_TEST_DEVICE_TIMEOUT 2u
 
 typedef struct {
   int32_t B, H, d;               /* d in {64, 128} */

@@ -19,9 +19,10 @@ constexpr int kKinds = 5;  // state, complement, attention, fold+ring, layout/pr
 enum Kind { K_STATE = 0, K_COMPLEMENT = 1, K_ATTN = 2, K_FOLD = 3, K_PREP = 4 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int32_t nseg_pad64(int32_t n) { return (n + 63) / 64 * 64; }
 
 struct Plan {
-  size_t status = 0, work = 0, entries = 0, pairs = 0, cm = 0, sseg = 0, srest = 0, srest_bf16 = 0;
+  size_t status = 0, work = 0, entries = 0, pairs = 0, cm = 0, cm_bf16 = 0, sseg = 0, srest = 0, srest_bf16 = 0;
   size_t ring_k = 0, ring_v = 0, mask = 0, total = 0;
   int64_t n_work = 0, n_entries = 0;
 };
@@ -50,6 +51,8 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
     p.mask = take(size_t(c.mask_heads) * nqt * nqt * nwc);
   } else {
     p.cm = take(sizeof(float) * size_t(L.cm_heads) * L.nqg * L.nseg);
+    if (c.mode == HYAT_MODE_BLOCKMASK || c.mode == HYAT_MODE_RADIAL)
+      p.cm_bf16 = take(2 * size_t(L.cm_heads) * L.nqg * nseg_pad64(L.nseg));
     p.sseg = take(sizeof(float) * BH * L.nseg * E);
     p.srest = take(sizeof(float) * BH * L.nqg * E);
     p.srest_bf16 = take(2 * BH * L.nqg * c.d * c.d);
@@ -99,6 +102,8 @@ struct hyat_ctx {
   int4* d_pairs = nullptr;
   int32_t n_pairs = 0;
   float* d_cm = nullptr;
+  uint16_t* d_cm_bf16 = nullptr;
+  bool use_gemm = false;             // tensor-core complement (block masks)
   float* d_sseg = nullptr;
   float* d_srest = nullptr;
   uint16_t* d_srest_bf16 = nullptr;
@@ -181,6 +186,7 @@ AttnArgs attn_args(hyat_ctx* h, const void* q, const void* k, const void* v, voi
   const float scale = h->cfg.scale > 0.0f ? h->cfg.scale : 1.0f / std::sqrt(float(h->cfg.d));
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = h->d_status;
+  a.test_timeout = (h->cfg.flags & HYAT_FLAG_TEST_DEVICE_TIMEOUT) ? 1 : 0;
   return a;
 }
 
@@ -262,6 +268,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
     h->d_mask = reinterpret_cast<uint8_t*>(ws + h->plan.mask);
   } else {
     h->d_cm = reinterpret_cast<float*>(ws + h->plan.cm);
+    if (h->plan.cm_bf16) h->d_cm_bf16 = reinterpret_cast<uint16_t*>(ws + h->plan.cm_bf16);
     h->d_sseg = reinterpret_cast<float*>(ws + h->plan.sseg);
   }
 
@@ -275,6 +282,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   }
   h->use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
               attn_tc_supported(cfg->d, cfg->dtype);
+  h->use_gemm = h->use_tc && h->d_cm_bf16 != nullptr && complement_tc_supported(cfg->d, h->lay.nqg);
 
   // layout tables and zeroed state
   e = cudaMemset(ws, 0, h->plan.status + 256);
@@ -291,6 +299,17 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
     e = cudaMemcpy(h->d_pairs, pairs.data(), sizeof(int4) * pairs.size(), cudaMemcpyHostToDevice);
   if (e == cudaSuccess && !h->lay.cm.empty())
     e = cudaMemcpy(h->d_cm, h->lay.cm.data(), sizeof(float) * h->lay.cm.size(), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && h->d_cm_bf16) {
+    // the 0/1 complement matrix as bf16 (exact), rows padded to a multiple of 64 segments
+    const int32_t np = nseg_pad64(h->lay.nseg);
+    std::vector<uint16_t> cmb(size_t(h->lay.cm_heads) * h->lay.nqg * np, 0);
+    for (int32_t m = 0; m < h->lay.cm_heads; ++m)
+      for (int32_t g = 0; g < h->lay.nqg; ++g)
+        for (int32_t sg = 0; sg < h->lay.nseg; ++sg)
+          if (h->lay.cm[(size_t(m) * h->lay.nqg + g) * h->lay.nseg + sg] != 0.0f)
+            cmb[(size_t(m) * h->lay.nqg + g) * np + sg] = 0x3F80;   // bf16 1.0
+    e = cudaMemcpy(h->d_cm_bf16, cmb.data(), 2 * cmb.size(), cudaMemcpyHostToDevice);
+  }
   if (e == cudaSuccess && cfg->mode == HYAT_MODE_STREAM)
     e = cudaMemset(ws + h->plan.srest, 0, h->plan.total - h->plan.srest);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -327,6 +346,10 @@ hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const vo
   sa.BH = h->BH; sa.d = h->cfg.d; sa.dtype = h->cfg.dtype;
   sa.nseg = L.nseg; sa.seg_base = 0; sa.seg_stride = L.seg_stride; sa.seg_len = L.seg_len;
   sa.out = h->d_sseg; sa.accumulate = 0; sa.status = h->d_status;
+  if (h->use_gemm) {        // hi/lo bf16 parts for the tensor-core complement, in the same bytes
+    sa.out_hi = reinterpret_cast<uint16_t*>(h->d_sseg);
+    sa.out_lo = sa.out_hi + size_t(h->BH) * L.nseg * h->E;
+  }
   cudaError_t e = timed(h, K_STATE, s, [&] {
     return h->use_tc ? launch_seg_state_tc(sa, h->num_sms, s) : launch_seg_state(sa, s);
   });
@@ -337,7 +360,20 @@ hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const vo
   ca.write_f32_s = h->use_tc ? 0 : 1;       // the tensor-core path reads S as bf16, z as fp32
   ca.BH = h->BH; ca.H = h->cfg.H; ca.cm_heads = L.cm_heads; ca.nseg = L.nseg; ca.nqg = L.nqg; ca.E = h->E;
   ca.d = h->cfg.d;
-  e = timed(h, K_COMPLEMENT, s, [&] { return launch_complement(ca, s); });
+  if (h->use_gemm) {
+    ComplementTcArgs ga{};
+    ga.cm_bf16 = h->d_cm_bf16;
+    ga.seg_hi = sa.out_hi;
+    ga.seg_lo = sa.out_lo;
+    ga.srest = h->d_srest;
+    ga.srest_bf16 = h->d_srest_bf16;
+    ga.write_f32_s = 0;
+    ga.BH = h->BH; ga.H = h->cfg.H; ga.mask_heads = L.cm_heads; ga.nqg = L.nqg; ga.nseg = L.nseg;
+    ga.nseg_pad = nseg_pad64(L.nseg); ga.E = h->E; ga.status = h->d_status;
+    e = timed(h, K_COMPLEMENT, s, [&] { return launch_complement_tc(ga, h->num_sms, s); });
+  } else {
+    e = timed(h, K_COMPLEMENT, s, [&] { return launch_complement(ca, s); });
+  }
   if (e != cudaSuccess) return cuda_fail(h, e, "complement kernel");
   return launch_attention(h, attn_args(h, q, k, v, o, h->plan.n_work, L.nqg), s);
 }

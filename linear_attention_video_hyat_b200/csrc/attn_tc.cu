@@ -67,7 +67,8 @@ struct __align__(1024) Smem {
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort_flag;
-  float z[2][D];                 // z_rest of each slot's current query tile
+  uint64_t never;                // test hook: a barrier nothing arrives on
+  unsigned long long timeout_ns; // limit of every bounded wait
 };
 
 struct TcParams {
@@ -81,6 +82,7 @@ struct TcParams {
   int32_t nqg;
   float scale_log2;
   uint32_t* status;
+  int32_t test_timeout;    // test hook: wait once on a barrier nothing signals (20 ms limit)
 };
 
 // Bounded wait on a phase parity. Returns false if the kernel is aborting.
@@ -91,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Smem* sm
     if (mbar_try_wait(b, parity)) return true;
     if ((it & 63u) == 0) {
       if (*reinterpret_cast<volatile int32_t*>(&sm->abort_flag)) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
+      if (globaltimer() - t0 > sm->timeout_ns) {
         atomicOr(status, kStatusTimeout);
         *reinterpret_cast<volatile int32_t*>(&sm->abort_flag) = 1;
         return false;
@@ -158,12 +160,11 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
     if (!wait_warp(q_full, qph, sm, p.status)) return;
     qph ^= 1u;
     // phi(q) of this row -> TMEM (bf16 pairs), l = phi(q) . z
-    // z_rest of this tile's group into shared memory: one coalesced load per warpgroup
-    const float* zg = p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D;
-    float* z = sm->z[s];
-    asm volatile("bar.sync %0, 128;" ::"r"(1 + s) : "memory");       // previous readers are done
-    z[row] = __ldg(zg + row);
-    asm volatile("bar.sync %0, 128;" ::"r"(1 + s) : "memory");
+    // z_rest of this tile's group: each lane holds 4 values (one coalesced 512-byte load per
+    // warp) and the phi loop broadcasts them with shuffles
+    const float4 zq = __ldg(reinterpret_cast<const float4*>(
+        p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D) + (row & 31));
+    const float zreg[4] = {zq.x, zq.y, zq.z, zq.w};
     float l = 0.0f, m = 0.0f;
     {
       const uint8_t* qrow = sm->q[s] + row * 128;
@@ -171,9 +172,9 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
 #pragma unroll 4
       for (int c = 0; c < 16; ++c) {            // 8 columns per step
         const uint4 raw = *reinterpret_cast<const uint4*>(qrow + (c >> 3) * HALF_BYTES + (((c & 7) ^ (row & 7)) << 4));
-        const float4 za = *reinterpret_cast<const float4*>(z + 8 * c);
-        const float4 zb = *reinterpret_cast<const float4*>(z + 8 * c + 4);
-        const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+        float zz[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) zz[t] = __shfl_sync(0xffffffffu, zreg[t & 3], 2 * c + (t >> 2));
         const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
         uint32_t pk[4];
 #pragma unroll
@@ -191,6 +192,7 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
       tc_fence_before();
       mbar_arrive(p_full);
     }
+    if (p.test_timeout && !wait_warp(&sm->never, 0, sm, p.status)) return;
     for (int j = 0; j < n; ++j) {
       const int klen = klen_next;
       if (j + 1 < n) klen_next = ent[j + 1].k_len;
@@ -295,7 +297,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&sm->pv_done[s], 1);
     }
     mbar_init(&sm->drain, 1);
+    mbar_init(&sm->never, 1);
     sm->abort_flag = 0;
+    sm->timeout_ns = p.test_timeout ? 20000000ull : kTimeoutNs;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -538,6 +542,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s) {
   p.nqg = a.nqg;
   p.scale_log2 = a.scale_log2;
   p.status = a.status;
+  p.test_timeout = a.test_timeout;
   const int grid = a.n_pairs < num_sms ? a.n_pairs : num_sms;
   return launch_pdl(attn_tc_kernel, dim3(grid), dim3(NUM_THREADS), kSmemBytes, s, mq, mk, mv, ms, p);
 }

@@ -65,6 +65,8 @@ struct SegStateArgs {
   float* out;                 // [BH][nseg][E], E = d*d + d (S row-major [a][b], then z[a])
   int32_t accumulate;         // out += instead of out =
   uint32_t* status;           // device status word (tensor-core kernel's bounded waits)
+  uint16_t* out_hi;           // tensor-core kernel only: if set, write bf16 hi = bf16(x) and
+  uint16_t* out_lo;           // lo = bf16(x - hi) ([BH][nseg][E] each) instead of fp32 `out`
 };
 cudaError_t launch_seg_state(const SegStateArgs& a, cudaStream_t s);
 cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t s);
@@ -78,6 +80,21 @@ struct ComplementArgs {
   int32_t BH, H, cm_heads, nseg, nqg, E, d;
 };
 cudaError_t launch_complement(const ComplementArgs& a, cudaStream_t s);
+
+// Tensor-core complement for block masks (d = 128, more than 8 groups): a GEMM of the bf16
+// 0/1 complement matrix with the hi/lo bf16 segment states (gemm_tc.cu).
+struct ComplementTcArgs {
+  const uint16_t* cm_bf16;    // [mask_heads][nqg][nseg_pad] bf16 0/1, rows padded with zeros
+  const uint16_t* seg_hi;     // [BH][nseg][E]
+  const uint16_t* seg_lo;     // [BH][nseg][E]
+  float* srest;               // [BH][nqg][E]: z always; S only if write_f32_s
+  uint16_t* srest_bf16;       // [BH][nqg][d][d]
+  int32_t write_f32_s;
+  int32_t BH, H, mask_heads, nqg, nseg, nseg_pad, E;
+  uint32_t* status;
+};
+bool complement_tc_supported(int d, int nqg);
+cudaError_t launch_complement_tc(const ComplementTcArgs& a, int num_sms, cudaStream_t s);
 
 // S (fp32 [a][b], group stride d*d + d) -> bf16 S [a][b] (group stride d*d) for the
 // tensor-core linear term, where S in its natural layout is the MN-major B operand.
@@ -95,6 +112,7 @@ struct AttnArgs {
   int32_t nqg, d, dtype, BH;
   float scale_log2;           // scale * log2(e)
   uint32_t* status;
+  int32_t test_timeout;       // HYAT_FLAG_TEST_DEVICE_TIMEOUT (tensor-core path)
 };
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s);

@@ -56,6 +56,8 @@ struct StateParams {
   float* out;
   int32_t accumulate;
   uint32_t* status;
+  uint16_t* out_hi;          // if set: bf16 hi/lo parts instead of fp32 `out`
+  uint16_t* out_lo;
 };
 
 __device__ __forceinline__ bool swait(uint64_t* b, uint32_t parity, StateSmem* sm, uint32_t* status) {
@@ -243,7 +245,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
       if (!swait_warp(&sm->acc_full[buf], (c >> 1) & 1, sm, p.status)) break;
       tc_fence_after();
       const uint32_t tacc = tmem + buf * 256 + lane_off;
-      float* out = p.out + (static_cast<int64_t>(x.bh) * p.nseg + x.g) * (D * D + D);
+      const int64_t obase = (static_cast<int64_t>(x.bh) * p.nseg + x.g) * (D * D + D);
+      float* out = p.out + obase;
       uint32_t zr[1];
       asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(zr[0]) : "r"(tacc + 128));
 #pragma unroll 1
@@ -256,19 +259,46 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
           tc_fence_before();
           mbar_arrive(&sm->acc_empty[buf]);
         }
-        float4* dst = reinterpret_cast<float4*>(out + a * D + 64 * h);
+        if (p.out_hi) {
+          // hi = bf16(x), lo = bf16(x - hi): 16-byte stores of 8 values each
+          uint4* dhi = reinterpret_cast<uint4*>(p.out_hi + obase + a * D + 64 * h);
+          uint4* dlo = reinterpret_cast<uint4*>(p.out_lo + obase + a * D + 64 * h);
 #pragma unroll
-        for (int v = 0; v < 16; ++v) {
-          float4 val = make_float4(u2f(r[4 * v]), u2f(r[4 * v + 1]), u2f(r[4 * v + 2]), u2f(r[4 * v + 3]));
-          if (p.accumulate) {
-            const float4 o = dst[v];
-            val.x += o.x; val.y += o.y; val.z += o.z; val.w += o.w;
+          for (int v = 0; v < 8; ++v) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const float x0 = u2f(r[8 * v + 2 * t]), x1 = u2f(r[8 * v + 2 * t + 1]);
+              hw[t] = pack_bf16(x0, x1);
+              const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[t]));
+              lw[t] = pack_bf16(x0 - hf.x, x1 - hf.y);
+            }
+            dhi[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            dlo[v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
           }
-          dst[v] = val;
+        } else {
+          float4* dst = reinterpret_cast<float4*>(out + a * D + 64 * h);
+#pragma unroll
+          for (int v = 0; v < 16; ++v) {
+            float4 val = make_float4(u2f(r[4 * v]), u2f(r[4 * v + 1]), u2f(r[4 * v + 2]), u2f(r[4 * v + 3]));
+            if (p.accumulate) {
+              const float4 o = dst[v];
+              val.x += o.x; val.y += o.y; val.z += o.z; val.w += o.w;
+            }
+            dst[v] = val;
+          }
         }
       }
-      float* zp = out + D * D + a;
-      *zp = p.accumulate ? *zp + u2f(zr[0]) : u2f(zr[0]);
+      const float zv = u2f(zr[0]);
+      if (p.out_hi) {
+        const __nv_bfloat16 zh = __float2bfloat16_rn(zv);
+        const __nv_bfloat16 zl = __float2bfloat16_rn(zv - __bfloat162float(zh));
+        p.out_hi[obase + D * D + a] = *reinterpret_cast<const uint16_t*>(&zh);
+        p.out_lo[obase + D * D + a] = *reinterpret_cast<const uint16_t*>(&zl);
+      } else {
+        float* zp = out + D * D + a;
+        *zp = p.accumulate ? *zp + zv : zv;
+      }
     }
   }
 
@@ -308,6 +338,8 @@ cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t
   p.out = a.out;
   p.accumulate = a.accumulate;
   p.status = a.status;
+  p.out_hi = a.out_hi;
+  p.out_lo = a.out_lo;
   const int grid = p.n_units < num_sms ? p.n_units : num_sms;
   state_tc_kernel<<<grid, ST_THREADS, kStateSmemBytes, s>>>(mk, mv, p);
   return cudaGetLastError();

@@ -216,6 +216,26 @@ def test_invalid_calls_return_errors_and_handle_stays_usable():
     h.close()
 
 
+def test_device_timeout_is_reported_and_recoverable():
+    """The timeout path without faulting the GPU: a wait on a signal that never comes gives up
+    after 20 ms, the call reports HYAT_ERR_DEVICE_TIMEOUT, and later calls work."""
+    w = wl.Workload("timeout", "window", 1, 2, 128, 200, 4, 2, 1, seed=2)
+    q, k, v = _dev(*wl.gen_qkv(w))
+    h = hyat.Hyat(hyat.config_from_workload(w, flags=hyat.FLAG_TEST_DEVICE_TIMEOUT))
+    h.forward(q, k, v)
+    with pytest.raises(hyat.HyatError) as ei:
+        h.sync()
+    assert ei.value.status == hyat.ERR_DEVICE_TIMEOUT
+    h.sync()                                            # the status word was cleared
+    h.close()
+    h2 = hyat.Hyat(hyat.config_from_workload(w))
+    o = h2.forward(q, k, v)
+    h2.sync()
+    ref = _window_ref(w, *(t.cpu() for t in (q, k, v)))
+    assert_parity("bf16", f64(o.cpu()), ref, "after a device timeout")
+    h2.close()
+
+
 # ------------------------------------------------------------------ full-size workloads
 def _bidir_sampled(w, heads, per_tile=2, seed=0):
     o, (q, k, v) = _bidir(w)
