@@ -14,8 +14,9 @@
 //   * one persistent CTA per SM; a CTA owns a pair of 128-row query tiles
 //     ("slots"), so the softmax of one slot overlaps the MMAs of the other;
 //   * warp 8 issues TMA loads (Q tiles, K/V tiles, bf16 S_rest) into 128B-swizzled
-//     shared memory through a 5-stage ring; warp 9 issues tcgen05.mma (one
-//     thread) with fp32 accumulators in TMEM; warps 0-3 / 4-7 run the softmax
+//     shared memory through a 5-stage ring; warp 9 issues tcgen05.mma (the
+//     whole warp runs the role, one elected lane issues) with fp32 accumulators
+//     in TMEM; warps 0-3 / 4-7 run the softmax
 //     of slot 0 / 1, one query row per thread, reading S from TMEM and writing
 //     P (bf16) back into TMEM, where it is the A operand of the P.V MMA;
 //   * TMEM (512 columns): S0 | S1 | O0 | O1, each 128 columns; P and phi(Q)
@@ -85,19 +86,20 @@ struct TcParams {
   int32_t test_timeout;    // test hook: wait once on a barrier nothing signals (20 ms limit)
 };
 
-// Bounded wait on a phase parity. Returns false if the kernel is aborting.
+// Bounded wait on a phase parity. Returns false if the kernel is aborting. After the first
+// probe the thread lets the hardware suspend it until the phase completes (at most
+// kSuspendNs per try), so waiting warps do not poll shared memory.
+constexpr uint32_t kSuspendNs = 1000000;
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Smem* sm, uint32_t* status) {
   if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*reinterpret_cast<volatile int32_t*>(&sm->abort_flag)) return false;
-      if (globaltimer() - t0 > sm->timeout_ns) {
-        atomicOr(status, kStatusTimeout);
-        *reinterpret_cast<volatile int32_t*>(&sm->abort_flag) = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_suspend(b, parity, kSuspendNs)) return true;
+    if (*reinterpret_cast<volatile int32_t*>(&sm->abort_flag)) return false;
+    if (globaltimer() - t0 > sm->timeout_ns) {
+      atomicOr(status, kStatusTimeout);
+      *reinterpret_cast<volatile int32_t*>(&sm->abort_flag) = 1;
+      return false;
     }
   }
 }
@@ -377,19 +379,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-    } else if (warp == MMA_WARP && lane == 0) {
+    } else if (warp == MMA_WARP) {
+      // the whole warp runs this role (warp-uniform descriptors); one elected lane issues
       int st = 0;
       uint32_t ph = 0, qph0 = 0, qph1 = 0, pph0 = 0, pph1 = 0;
       bool ok = true;
       auto next_stage = [&](int& out) -> bool {
-        if (!mbar_wait(&sm->kv_full[st], ph, sm, p.status)) return false;
+        if (!mbar_wait_warp(&sm->kv_full[st], ph, sm, p.status)) return false;
         tc_fence_after();
         out = st;
         if (++st == NS) { st = 0; ph ^= 1u; }
         return true;
       };
       auto wait_p = [&](uint64_t* bar, uint32_t& phase) -> bool {
-        if (!mbar_wait(bar, phase, sm, p.status)) return false;
+        if (!mbar_wait_warp(bar, phase, sm, p.status)) return false;
         phase ^= 1u;
         tc_fence_after();
         return true;
@@ -405,20 +408,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto qk = [&](uint32_t tS, uint64_t dq, int stage, uint64_t* done) {
         const uint64_t dk = dK0 + static_cast<uint64_t>(stage) * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ss(tS, dq + koff(kk), dk + koff(kk), kIdescKK, kk > 0);
-        mma_commit(done);
+        for (int kk = 0; kk < 8; ++kk) mma_ss_elect(tS, dq + koff(kk), dk + koff(kk), kIdescKK, kk > 0);
+        mma_commit_elect(done);
       };
       auto pv = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
         const uint64_t dv = dV0 + static_cast<uint64_t>(stage) * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescKMN, 1);
-        mma_commit(done);
+        for (int kk = 0; kk < 8; ++kk) mma_ts_elect(tO, tS + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescKMN, 1);
+        mma_commit_elect(done);
       };
       auto linear = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
         const uint64_t dv = dV0 + static_cast<uint64_t>(stage) * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts(tO, tS + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescKMN, kk > 0);
-        mma_commit(done);
+        for (int kk = 0; kk < 8; ++kk) mma_ts_elect(tO, tS + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescKMN, kk > 0);
+        mma_commit_elect(done);
       };
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
       for (int pi = blockIdx.x; pi < p.n_pairs && ok; pi += gridDim.x) {
@@ -431,8 +434,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = wait_p(&sm->p_full[0], pph0) && next_stage(sst);
         if (!ok) break;
         linear(tO0, tS0, sst, &sm->pv_done[0]);
-        mma_commit(&sm->kv_empty[sst]);
-        ok = mbar_wait(&sm->q_full[0], qph0, sm, p.status);
+        mma_commit_elect(&sm->kv_empty[sst]);
+        ok = mbar_wait_warp(&sm->q_full[0], qph0, sm, p.status);
         if (!ok) break;
         qph0 ^= 1u;
         tc_fence_after();
@@ -440,16 +443,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = next_stage(k0);
           if (!ok) break;
           qk(tS0, dQ0, k0, &sm->s_full[0]);
-          if (!shared) mma_commit(&sm->kv_empty[k0]);
+          if (!shared) mma_commit_elect(&sm->kv_empty[k0]);
         }
-        if (n0 <= 1) mma_commit(&sm->q_empty[0]);
+        if (n0 <= 1) mma_commit_elect(&sm->q_empty[0]);
         // slot 1
         if (has1) {
           ok = wait_p(&sm->p_full[1], pph1) && next_stage(sst);
           if (!ok) break;
           linear(tO1, tS1, sst, &sm->pv_done[1]);
-          mma_commit(&sm->kv_empty[sst]);
-          ok = mbar_wait(&sm->q_full[1], qph1, sm, p.status);
+          mma_commit_elect(&sm->kv_empty[sst]);
+          ok = mbar_wait_warp(&sm->q_full[1], qph1, sm, p.status);
           if (!ok) break;
           qph1 ^= 1u;
           tc_fence_after();
@@ -457,21 +460,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (shared) k1 = k0;
             else if (!(ok = next_stage(k1))) break;
             qk(tS1, dQ1, k1, &sm->s_full[1]);
-            mma_commit(&sm->kv_empty[k1]);
+            mma_commit_elect(&sm->kv_empty[k1]);
           }
-          if (n1 <= 1) mma_commit(&sm->q_empty[1]);
+          if (n1 <= 1) mma_commit_elect(&sm->q_empty[1]);
         }
         const int nmax = n0 > n1 ? n0 : n1;
         for (int j = 0; j < nmax && ok; ++j) {
           if (j < n0) {
             if (!(ok = wait_p(&sm->p_full[0], pph0) && next_stage(v0))) break;
             pv(tO0, tS0, v0, &sm->pv_done[0]);
-            if (!shared) mma_commit(&sm->kv_empty[v0]);
+            if (!shared) mma_commit_elect(&sm->kv_empty[v0]);
             if (j + 1 < n0) {
               if (!(ok = next_stage(k0))) break;
               qk(tS0, dQ0, k0, &sm->s_full[0]);
-              if (!shared) mma_commit(&sm->kv_empty[k0]);
-              if (j + 2 == n0) mma_commit(&sm->q_empty[0]);
+              if (!shared) mma_commit_elect(&sm->kv_empty[k0]);
+              if (j + 2 == n0) mma_commit_elect(&sm->q_empty[0]);
             }
           }
           if (has1 && j < n1) {
@@ -479,22 +482,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (shared) v1 = v0;
             else if (!(ok = next_stage(v1))) break;
             pv(tO1, tS1, v1, &sm->pv_done[1]);
-            mma_commit(&sm->kv_empty[v1]);
+            mma_commit_elect(&sm->kv_empty[v1]);
             if (j + 1 < n1) {
               if (shared) k1 = k0;
               else if (!(ok = next_stage(k1))) break;
               qk(tS1, dQ1, k1, &sm->s_full[1]);
-              mma_commit(&sm->kv_empty[k1]);
-              if (j + 2 == n1) mma_commit(&sm->q_empty[1]);
+              mma_commit_elect(&sm->kv_empty[k1]);
+              if (j + 2 == n1) mma_commit_elect(&sm->q_empty[1]);
             }
           }
         }
       }
       // wait for every issued MMA before TMEM is released
-      mma_commit(&sm->drain);
+      mma_commit_elect(&sm->drain);
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(&sm->drain, 0) && globaltimer() - t0 < kTimeoutNs) {
       }
+      __syncwarp();
     }
   } else {
     // -------------------------------------------------------------- softmax warpgroups
