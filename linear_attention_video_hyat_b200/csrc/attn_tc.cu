@@ -467,25 +467,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int nmax = n0 > n1 ? n0 : n1;
         for (int j = 0; j < nmax && ok; ++j) {
           if (j < n0) {
-            if (!(ok = wait_p(&sm->p_full[0], pph0) && next_stage(v0))) break;
+            // the stage waits come first: they are usually satisfied while the softmax still
+            // runs, so once P lands the block issues with no wait in between
+            if (!(ok = next_stage(v0))) break;
+            if (j + 1 < n0 && !(ok = next_stage(k0))) break;
+            if (!(ok = wait_p(&sm->p_full[0], pph0))) break;
             pv(tO0, tS0, v0, &sm->pv_done[0]);
             if (!shared) mma_commit_elect(&sm->kv_empty[v0]);
             if (j + 1 < n0) {
-              if (!(ok = next_stage(k0))) break;
               qk(tS0, dQ0, k0, &sm->s_full[0]);
               if (!shared) mma_commit_elect(&sm->kv_empty[k0]);
               if (j + 2 == n0) mma_commit_elect(&sm->q_empty[0]);
             }
           }
           if (has1 && j < n1) {
+            if (shared) {
+              v1 = v0;
+              k1 = k0;
+            } else {
+              if (!(ok = next_stage(v1))) break;
+              if (j + 1 < n1 && !(ok = next_stage(k1))) break;
+            }
             if (!(ok = wait_p(&sm->p_full[1], pph1))) break;
-            if (shared) v1 = v0;
-            else if (!(ok = next_stage(v1))) break;
             pv(tO1, tS1, v1, &sm->pv_done[1]);
             mma_commit_elect(&sm->kv_empty[v1]);
             if (j + 1 < n1) {
-              if (shared) k1 = k0;
-              else if (!(ok = next_stage(k1))) break;
               qk(tS1, dQ1, k1, &sm->s_full[1]);
               mma_commit_elect(&sm->kv_empty[k1]);
               if (j + 2 == n1) mma_commit_elect(&sm->q_empty[1]);
