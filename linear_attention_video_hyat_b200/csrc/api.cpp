@@ -293,7 +293,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
                    cudaMemcpyHostToDevice);
   const std::vector<int4> pairs = cfg->mode == HYAT_MODE_STREAM
                                       ? build_stream_pairs(h->BH, tiles(stream_chunk_tokens(*cfg)))
-                                      : build_pairs(h->lay.work);
+                                      : order_pairs_for_grid(build_pairs(h->lay.work), h->lay.work, h->num_sms);
   h->n_pairs = static_cast<int32_t>(pairs.size());
   if (e == cudaSuccess && !pairs.empty())
     e = cudaMemcpy(h->d_pairs, pairs.data(), sizeof(int4) * pairs.size(), cudaMemcpyHostToDevice);

@@ -54,6 +54,10 @@ std::string build_layout(const hyat_config& c, const uint8_t* host_mask, Layout*
 // Pair consecutive work items of the same (b, h) into units of two query tiles;
 // `shared` marks pairs whose key lists are identical (loaded once for both).
 std::vector<int4> build_pairs(const std::vector<WorkItem>& work);
+// Reorder pairs so that a persistent grid of `grid` CTAs, taking pair k on CTA k mod grid,
+// gets nearly equal work: largest pairs first, dealt out in a serpentine order.
+std::vector<int4> order_pairs_for_grid(const std::vector<int4>& pairs, const std::vector<WorkItem>& work,
+                                       int32_t grid);
 std::vector<int4> build_stream_pairs(int32_t BH, int32_t nqt);
 void radial_tile_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t* out);
 

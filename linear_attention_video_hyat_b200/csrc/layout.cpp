@@ -213,6 +213,28 @@ std::vector<int4> build_pairs(const std::vector<WorkItem>& work) {
   return pairs;
 }
 
+std::vector<int4> order_pairs_for_grid(const std::vector<int4>& pairs, const std::vector<WorkItem>& work,
+                                       int32_t grid) {
+  if (grid <= 1 || pairs.size() <= static_cast<size_t>(grid)) return pairs;
+  // cost of a pair: its key tiles (both slots) plus two tiles' worth of per-pair set-up
+  auto n_of = [&](int item) { return item < 0 ? 0 : work[item].entry_end - work[item].entry_begin; };
+  std::vector<int64_t> cost(pairs.size());
+  for (size_t i = 0; i < pairs.size(); ++i) cost[i] = n_of(pairs[i].x) + n_of(pairs[i].y) + 2;
+  std::vector<size_t> idx(pairs.size());
+  for (size_t i = 0; i < idx.size(); ++i) idx[i] = i;
+  std::stable_sort(idx.begin(), idx.end(), [&](size_t a, size_t b) { return cost[a] > cost[b]; });
+  // The kernel hands pair k to CTA k mod grid. Placing the pairs largest first in rows of
+  // `grid`, with every other row reversed, deals them out in a serpentine order.
+  std::vector<int4> out(pairs.size());
+  for (size_t k = 0; k < idx.size(); ++k) {
+    const size_t row = k / grid, col = k % grid;
+    const size_t row_len = std::min<size_t>(grid, idx.size() - row * grid);
+    const size_t c = (row & 1) ? row_len - 1 - col : col;
+    out[row * grid + c] = pairs[idx[k]];
+  }
+  return out;
+}
+
 std::vector<int4> build_stream_pairs(int32_t BH, int32_t nqt) {
   std::vector<int4> pairs;
   for (int32_t bh = 0; bh < BH; ++bh)

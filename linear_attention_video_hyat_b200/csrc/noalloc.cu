@@ -70,7 +70,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
 
   Layout L;
   if (!build_layout(*cfg, nullptr, &L).empty()) return HYAT_ERR_INVALID_ARG;
-  const std::vector<int4> pairs = build_pairs(L.work);
+  std::vector<int4> pairs = build_pairs(L.work);
   const int64_t BH = int64_t(cfg->B) * cfg->H;
   const int64_t E = int64_t(cfg->d) * cfg->d + cfg->d;
   const int64_t rows = rows_q(*cfg);
@@ -91,6 +91,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   void* base = nullptr;
   int num_sms = 0;
   if (scratch_for_current_device(&base, &num_sms) != cudaSuccess) return HYAT_ERR_CUDA;
+  pairs = order_pairs_for_grid(pairs, L.work, num_sms);
   char* ws = static_cast<char*>(base);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
