@@ -138,6 +138,19 @@ HYAT_API hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k,
 HYAT_API hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, const void* v,
                                  void* o, const uint8_t* host_step_mask, void* stream);
 
+/* A non-final call for the current streaming chunk: one denoising step of it.
+ * Streaming video models denoise a chunk in several calls and keep only the
+ * last call's keys and values in the cache (Hybrid Forcing, Section 2.A: the
+ * window holds the frames already generated). A chunk's calls are any number
+ * of hyat_fwd_stream_denoise calls followed by one hyat_fwd_stream_step,
+ * which is the final call and advances the step counter. Every call sees the
+ * committed window chunks, the folded state and its own Q, K, V as the
+ * newest chunk; arguments, layouts and the mask are those of
+ * hyat_fwd_stream_step. The chunk leaving the window is folded once, at the
+ * chunk's first call. */
+HYAT_API hyat_status hyat_fwd_stream_denoise(hyat_handle h, const void* q, const void* k, const void* v,
+                                    void* o, const uint8_t* host_step_mask, void* stream);
+
 /* Wait for the last call's stream and report device-side errors. */
 HYAT_API hyat_status hyat_sync(hyat_handle h);
 
@@ -169,7 +182,9 @@ HYAT_API hyat_status hyat_radial_mask(int32_t n_frames, int32_t tokens_per_frame
 HYAT_API hyat_status hyat_stream_plan(const hyat_config* cfg, int32_t step, int32_t* info,
                              size_t info_len);
 
-/* Stream state (S, z, KV ring, step) to / from a host buffer. The size is
+/* Stream state (S, z, KV ring, step, and whether the current chunk's fold
+ * has run) to / from a host buffer: a 48-byte header, then S, z as fp32
+ * [B*H][d*d + d], then the K and V rings. The size is
  * hyat_stream_state_bytes(); both calls synchronise the device. */
 HYAT_API size_t hyat_stream_state_bytes(hyat_handle h);
 HYAT_API hyat_status hyat_stream_get_state(hyat_handle h, void* dst_host, size_t bytes);

@@ -23,11 +23,22 @@ int32_t nseg_pad64(int32_t n) { return (n + 63) / 64 * 64; }
 
 struct Plan {
   size_t status = 0, work = 0, entries = 0, pairs = 0, cm = 0, cm_bf16 = 0, sseg = 0, srest = 0, srest_bf16 = 0;
-  size_t ring_k = 0, ring_v = 0, mask = 0, total = 0;
+  size_t ring_k = 0, ring_v = 0, mask = 0, fold_partial = 0, total = 0;
   int64_t n_work = 0, n_entries = 0;
 };
 
 int64_t elem_bytes(const hyat_config& c) { return c.dtype == HYAT_F32 ? 4 : 2; }
+
+// The streaming fold splits the evicted chunk of every (b, h) into token ranges so that the
+// state kernel fills the GPU (one range per SM, about); the workspace holds up to
+// kFoldPartsMax ranges per (b, h), enough for 256 SMs.
+constexpr int32_t kFoldPartsMax = 32;
+int32_t fold_parts_cap(const hyat_config& c) {
+  const int64_t BH = int64_t(c.B) * c.H;
+  const int64_t by_sms = std::max<int64_t>(1, 256 / std::max<int64_t>(BH, 1));
+  const int64_t by_len = (stream_chunk_tokens(c) + 127) / 128;
+  return static_cast<int32_t>(std::min<int64_t>({by_sms, by_len, kFoldPartsMax}));
+}
 
 // Offsets of every region in the caller's workspace.
 Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const Layout& L) {
@@ -49,6 +60,7 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
     p.ring_k = take(size_t(BH * nwc * Lc * c.d * elem_bytes(c)));
     p.ring_v = take(size_t(BH * nwc * Lc * c.d * elem_bytes(c)));
     p.mask = take(size_t(c.mask_heads) * nqt * nqt * nwc);
+    p.fold_partial = take(sizeof(float) * BH * fold_parts_cap(c) * E);
   } else {
     p.cm = take(sizeof(float) * size_t(L.cm_heads) * L.nqg * L.nseg);
     if (c.mode == HYAT_MODE_BLOCKMASK || c.mode == HYAT_MODE_RADIAL)
@@ -111,6 +123,9 @@ struct hyat_ctx {
   void* d_ring_v = nullptr;
   uint8_t* d_mask = nullptr;
   int32_t step = 0;
+  int32_t folded_step = -1;          // step whose evicted chunk is already in S, z
+  float* d_fold_partial = nullptr;
+  int32_t fold_parts = 1, fold_part_len = 0;
   bool use_tc = false;
   int num_sms = 148;
   cudaStream_t last_stream = nullptr;
@@ -266,6 +281,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
     h->d_ring_k = ws + h->plan.ring_k;
     h->d_ring_v = ws + h->plan.ring_v;
     h->d_mask = reinterpret_cast<uint8_t*>(ws + h->plan.mask);
+    h->d_fold_partial = reinterpret_cast<float*>(ws + h->plan.fold_partial);
   } else {
     h->d_cm = reinterpret_cast<float*>(ws + h->plan.cm);
     if (h->plan.cm_bf16) h->d_cm_bf16 = reinterpret_cast<uint16_t*>(ws + h->plan.cm_bf16);
@@ -283,6 +299,14 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   h->use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
               attn_tc_supported(cfg->d, cfg->dtype);
   h->use_gemm = h->use_tc && h->d_cm_bf16 != nullptr && complement_tc_supported(cfg->d, h->lay.nqg);
+  if (cfg->mode == HYAT_MODE_STREAM) {
+    // token ranges of the fold: about one per SM, whole 64-token stages
+    const int32_t Lc = stream_chunk_tokens(*cfg);
+    const int32_t want = std::max<int32_t>(1, std::min<int32_t>(fold_parts_cap(*cfg), h->num_sms / std::max(h->BH, 1)));
+    const int32_t stages = (Lc + 63) / 64;
+    h->fold_part_len = (stages + want - 1) / want * 64;
+    h->fold_parts = (Lc + h->fold_part_len - 1) / h->fold_part_len;
+  }
 
   // layout tables and zeroed state
   e = cudaMemset(ws, 0, h->plan.status + 256);
@@ -378,8 +402,14 @@ hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const vo
   return launch_attention(h, attn_args(h, q, k, v, o, h->plan.n_work, L.nqg), s);
 }
 
-hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, const void* v, void* o,
-                                 const uint8_t* host_step_mask, void* stream) {
+namespace {
+
+// One streaming call for the current chunk. The first call of a chunk folds the chunk that
+// leaves the window into S, z; every call writes its K, V into the chunk's ring slot and
+// attends. `commit` marks the chunk's final call: the step counter then advances, and the
+// K, V just written stay in the window.
+hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void* v, void* o,
+                        const uint8_t* host_step_mask, void* stream, bool commit) {
   if (!h) return HYAT_ERR_INVALID_ARG;
   if (h->cfg.mode != HYAT_MODE_STREAM) return fail(h, HYAT_ERR_INVALID_ARG, "handle is not in STREAM mode");
   hyat_status st = check_ptrs(h, q, k, v, o);
@@ -406,17 +436,26 @@ hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, co
     e = cudaMemsetAsync(h->d_mask, 1, mask_bytes, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "step mask upload");
   const int32_t slot = s_ % nwc;
+  const bool fold = s_ >= nwc && h->folded_step != s_;
   e = timed(h, K_FOLD, s, [&]() -> cudaError_t {
-    if (s_ >= nwc) {  // chunk s - nwc leaves the window: fold it into S, z
+    if (fold) {  // chunk s - nwc leaves the window: fold it into S, z
       SegStateArgs sa{};
       sa.k = h->d_ring_k; sa.v = h->d_ring_v; sa.rows_per_bh = h->rk;
       sa.BH = h->BH; sa.d = c.d; sa.dtype = c.dtype;
       sa.nseg = 1; sa.seg_base = slot * Lc; sa.seg_stride = Lc; sa.seg_len = Lc;
       sa.out = h->d_srest; sa.accumulate = 1; sa.status = h->d_status;
-      cudaError_t e2 = h->use_tc ? launch_seg_state_tc(sa, h->num_sms, s) : launch_seg_state(sa, s);
-      if (e2 != cudaSuccess) return e2;
       if (h->use_tc) {
-        e2 = launch_state_to_bf16(h->d_srest, h->d_srest_bf16, h->BH, c.d, s);
+        // token ranges in parallel, then an ordered sum into S, z and the bf16 copy
+        sa.parts = h->fold_parts; sa.part_len = h->fold_part_len; sa.partial = h->d_fold_partial;
+        cudaError_t e2 = launch_seg_state_tc(sa, h->num_sms, s);
+        if (e2 != cudaSuccess) return e2;
+        FoldReduceArgs fa{};
+        fa.partial = h->d_fold_partial; fa.srest = h->d_srest; fa.srest_bf16 = h->d_srest_bf16;
+        fa.BH = h->BH; fa.parts = h->fold_parts; fa.d = c.d;
+        e2 = launch_fold_reduce(fa, s);
+        if (e2 != cudaSuccess) return e2;
+      } else {
+        cudaError_t e2 = launch_seg_state(sa, s);
         if (e2 != cudaSuccess) return e2;
       }
     }
@@ -427,6 +466,7 @@ hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, co
     return launch_ring_copy(ra, s);
   });
   if (e != cudaSuccess) return cuda_fail(h, e, "stream fold / ring copy");
+  if (fold) h->folded_step = s_;
   StreamLayoutArgs la{};
   la.mask = h->d_mask; la.work = h->d_work; la.entries = h->d_entries;
   la.BH = h->BH; la.H = c.H; la.mask_heads = c.mask_heads; la.nqt = nqt; la.nkt = nkt;
@@ -435,8 +475,20 @@ hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, co
   if (e != cudaSuccess) return cuda_fail(h, e, "stream layout kernel");
   st = launch_attention(h, attn_args(h, q, h->d_ring_k, h->d_ring_v, o, int64_t(h->BH) * nqt, 1), s);
   if (st != HYAT_OK) return st;
-  h->step += 1;
+  if (commit) h->step += 1;
   return HYAT_OK;
+}
+
+}  // namespace
+
+hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, const void* v, void* o,
+                                 const uint8_t* host_step_mask, void* stream) {
+  return stream_call(h, q, k, v, o, host_step_mask, stream, true);
+}
+
+hyat_status hyat_fwd_stream_denoise(hyat_handle h, const void* q, const void* k, const void* v, void* o,
+                                    const uint8_t* host_step_mask, void* stream) {
+  return stream_call(h, q, k, v, o, host_step_mask, stream, false);
 }
 
 hyat_status hyat_sync(hyat_handle h) {
@@ -497,6 +549,7 @@ namespace {
 struct StateHeader {
   uint32_t magic, version;
   int32_t step, BH, d, L, nwc, dtype;
+  int32_t folded_step, reserved[3];   // version 2: the step whose evicted chunk is in S, z
 };
 constexpr uint32_t kMagic = 0x54415948u;  // "HYAT"
 }  // namespace
@@ -514,8 +567,8 @@ hyat_status hyat_stream_get_state(hyat_handle h, void* dst_host, size_t bytes) {
   if (bytes < hyat_stream_state_bytes(h)) return fail(h, HYAT_ERR_INVALID_ARG, "state buffer too small");
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(h, e, "synchronize");
-  StateHeader hd{kMagic, 1, h->step, h->BH, h->cfg.d, stream_chunk_tokens(h->cfg), stream_window_chunks(h->cfg),
-                 h->cfg.dtype};
+  StateHeader hd{kMagic, 2, h->step, h->BH, h->cfg.d, stream_chunk_tokens(h->cfg), stream_window_chunks(h->cfg),
+                 h->cfg.dtype, h->folded_step, {0, 0, 0}};
   char* p = static_cast<char*>(dst_host);
   std::memcpy(p, &hd, sizeof(hd));
   p += sizeof(hd);
@@ -534,9 +587,9 @@ hyat_status hyat_stream_set_state(hyat_handle h, const void* src_host, size_t by
   if (bytes < hyat_stream_state_bytes(h)) return fail(h, HYAT_ERR_STATE, "state buffer too small");
   StateHeader hd;
   std::memcpy(&hd, src_host, sizeof(hd));
-  if (hd.magic != kMagic || hd.version != 1 || hd.BH != h->BH || hd.d != h->cfg.d ||
+  if (hd.magic != kMagic || hd.version != 2 || hd.BH != h->BH || hd.d != h->cfg.d ||
       hd.L != stream_chunk_tokens(h->cfg) || hd.nwc != stream_window_chunks(h->cfg) || hd.dtype != h->cfg.dtype ||
-      hd.step < 0)
+      hd.step < 0 || hd.folded_step > hd.step)
     return fail(h, HYAT_ERR_STATE, "state blob does not match this handle");
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(h, e, "synchronize");
@@ -550,6 +603,7 @@ hyat_status hyat_stream_set_state(hyat_handle h, const void* src_host, size_t by
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(h, e, "state copy");
   h->step = hd.step;
+  h->folded_step = hd.folded_step;
   return HYAT_OK;
 }
 

@@ -71,8 +71,24 @@ struct SegStateArgs {
   uint32_t* status;           // device status word (tensor-core kernel's bounded waits)
   uint16_t* out_hi;           // tensor-core kernel only: if set, write bf16 hi = bf16(x) and
   uint16_t* out_lo;           // lo = bf16(x - hi) ([BH][nseg][E] each) instead of fp32 `out`
+  // tensor-core kernel only: split each segment into `parts` token ranges of `part_len`
+  // tokens (a multiple of 64); the state of range r of segment g of bh goes to
+  // partial[((bh * nseg + g) * parts + r) * E] (plain store), and `out` is not written.
+  int32_t parts;
+  int32_t part_len;
+  float* partial;
 };
 cudaError_t launch_seg_state(const SegStateArgs& a, cudaStream_t s);
+
+// Streaming fold, second half: srest[bh] += sum over r of partial[bh][r] (fixed order, so the
+// result is deterministic), and the bf16 copy of S for the attention kernel.
+struct FoldReduceArgs {
+  const float* partial;       // [BH][parts][E]
+  float* srest;               // [BH][E]
+  uint16_t* srest_bf16;       // [BH][d][d]
+  int32_t BH, parts, d;
+};
+cudaError_t launch_fold_reduce(const FoldReduceArgs& a, cudaStream_t s);
 cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t s);
 
 struct ComplementArgs {

@@ -167,6 +167,32 @@ __global__ void state_to_bf16_kernel(const float* __restrict__ s, uint16_t* __re
   }
 }
 
+// srest[bh] += sum_r partial[bh][r], in order r = 0, 1, ...; then bf16(S) for the attention
+// kernel. One thread per 4 consecutive floats of a state.
+__global__ void fold_reduce_kernel(FoldReduceArgs a) {
+  const int64_t E4 = (static_cast<int64_t>(a.d) * a.d + a.d) / 4, dd4 = static_cast<int64_t>(a.d) * a.d / 4;
+  const int64_t total = E4 * a.BH;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t bh = i / E4, e4 = i % E4;
+    float4* dst = reinterpret_cast<float4*>(a.srest) + bh * E4 + e4;
+    float4 acc = *dst;
+    const float4* src = reinterpret_cast<const float4*>(a.partial) + bh * a.parts * E4 + e4;
+    for (int r = 0; r < a.parts; ++r) {
+      const float4 v = src[r * E4];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    *dst = acc;
+    if (e4 < dd4) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 w;
+      w.x = *reinterpret_cast<const uint32_t*>(&lo);
+      w.y = *reinterpret_cast<const uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(a.srest_bf16)[bh * dd4 + e4] = w;
+    }
+  }
+}
+
 // new chunk K/V -> ring slot, 16-byte vectors
 __global__ void ring_copy_kernel(RingCopyArgs a) {
   const int64_t row_vecs = static_cast<int64_t>(a.L) * a.d * a.elem_bytes / 16;
@@ -445,6 +471,15 @@ cudaError_t launch_state_to_bf16(const float* srest, uint16_t* out, int64_t n_gr
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s) {
   if (a.dtype == HYAT_F32) return a.d == 64 ? launch_attn_simt_t<float, 64>(a, s) : launch_attn_simt_t<float, 128>(a, s);
   return a.d == 64 ? launch_attn_simt_t<__nv_bfloat16, 64>(a, s) : launch_attn_simt_t<__nv_bfloat16, 128>(a, s);
+}
+
+cudaError_t launch_fold_reduce(const FoldReduceArgs& a, cudaStream_t s) {
+  const int64_t total = (static_cast<int64_t>(a.d) * a.d + a.d) / 4 * a.BH;
+  if (total == 0) return cudaSuccess;
+  if (a.d % 4 != 0) return cudaErrorInvalidValue;
+  const int blocks = static_cast<int>((total + 255) / 256 < 2048 ? (total + 255) / 256 : 2048);
+  fold_reduce_kernel<<<blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_ring_copy(const RingCopyArgs& a, cudaStream_t s) {

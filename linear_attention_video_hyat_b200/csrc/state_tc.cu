@@ -52,6 +52,8 @@ struct __align__(1024) StateSmem {
 
 struct StateParams {
   int32_t nseg, n_units, seg_base, seg_stride, seg_len;
+  int32_t parts, part_len;   // each segment is split into `parts` token ranges of part_len
+  float* partial;            // if set: unit u's state -> partial[u] (fp32, plain store)
   int64_t rows;
   float* out;
   int32_t accumulate;
@@ -85,13 +87,20 @@ struct Unit {
   int bh, g, start, len, ntiles;
 };
 
+// Unit u covers part (u mod parts) of segment (u / parts): tokens
+// [start, start + len) of (b, h) row block bh.
 __device__ __forceinline__ Unit unit_of(const StateParams& p, int u) {
   Unit x;
-  x.bh = u / p.nseg;
-  x.g = u % p.nseg;
-  x.start = p.seg_base + x.g * p.seg_stride;
+  const int su = u / p.parts, part = u - su * p.parts;
+  x.bh = su / p.nseg;
+  x.g = su % p.nseg;
+  const int off = part * p.part_len;
+  x.start = p.seg_base + x.g * p.seg_stride + off;
+  int len = p.seg_len - off;
+  if (len > p.part_len) len = p.part_len;
+  if (len < 0) len = 0;
   const int64_t rem = p.rows - x.start;
-  x.len = static_cast<int>(rem < p.seg_len ? (rem > 0 ? rem : 0) : p.seg_len);
+  x.len = static_cast<int>(rem < len ? (rem > 0 ? rem : 0) : len);
   x.ntiles = x.len > 0 ? (x.len + TOK - 1) / TOK : 1;
   return x;
 }
@@ -246,7 +255,8 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
       tc_fence_after();
       const uint32_t tacc = tmem + buf * 256 + lane_off;
       const int64_t obase = (static_cast<int64_t>(x.bh) * p.nseg + x.g) * (D * D + D);
-      float* out = p.out + obase;
+      float* out = p.partial ? p.partial + static_cast<int64_t>(u) * (D * D + D) : p.out + obase;
+      const bool acc_out = p.accumulate && !p.partial;
       uint32_t zr[1];
       asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(zr[0]) : "r"(tacc + 128));
 #pragma unroll 1
@@ -281,7 +291,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
 #pragma unroll
           for (int v = 0; v < 16; ++v) {
             float4 val = make_float4(u2f(r[4 * v]), u2f(r[4 * v + 1]), u2f(r[4 * v + 2]), u2f(r[4 * v + 3]));
-            if (p.accumulate) {
+            if (acc_out) {
               const float4 o = dst[v];
               val.x += o.x; val.y += o.y; val.z += o.z; val.w += o.w;
             }
@@ -297,7 +307,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
         p.out_lo[obase + D * D + a] = *reinterpret_cast<const uint16_t*>(&zl);
       } else {
         float* zp = out + D * D + a;
-        *zp = p.accumulate ? *zp + zv : zv;
+        *zp = acc_out ? *zp + zv : zv;
       }
     }
   }
@@ -328,9 +338,14 @@ cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  const int parts = a.parts > 1 ? a.parts : 1;
+  if (parts > 1 && (a.partial == nullptr || a.out_hi != nullptr || a.part_len <= 0)) return cudaErrorInvalidValue;
   StateParams p{};
   p.nseg = a.nseg;
-  p.n_units = a.nseg * a.BH;
+  p.parts = parts;
+  p.part_len = parts > 1 ? a.part_len : a.seg_len;
+  p.partial = parts > 1 ? a.partial : nullptr;
+  p.n_units = a.nseg * a.BH * parts;
   p.seg_base = a.seg_base;
   p.seg_stride = a.seg_stride;
   p.seg_len = a.seg_len;

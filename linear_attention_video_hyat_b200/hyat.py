@@ -31,7 +31,7 @@ EXPORTED = (
     "hyat_workspace_bytes", "hyat_create", "hyat_fwd_bidir", "hyat_fwd_stream_step", "hyat_sync",
     "hyat_destroy", "hyat_last_error", "hyat_status_string", "hyat_plan_layout", "hyat_radial_mask",
     "hyat_stream_plan", "hyat_stream_state_bytes", "hyat_stream_get_state", "hyat_stream_set_state",
-    "hyat_set_profiling", "hyat_kernel_times", "hyat_fwd_bidir_noalloc",
+    "hyat_set_profiling", "hyat_kernel_times", "hyat_fwd_bidir_noalloc", "hyat_fwd_stream_denoise",
 )
 
 
@@ -64,6 +64,7 @@ def _load():
         "hyat_create": (ctypes.c_int, [CP, P, S, P, ctypes.POINTER(P)]),
         "hyat_fwd_bidir": (ctypes.c_int, [P, P, P, P, P, P]),
         "hyat_fwd_stream_step": (ctypes.c_int, [P, P, P, P, P, P, P]),
+        "hyat_fwd_stream_denoise": (ctypes.c_int, [P, P, P, P, P, P, P]),
         "hyat_sync": (ctypes.c_int, [P]),
         "hyat_destroy": (ctypes.c_int, [P]),
         "hyat_last_error": (ctypes.c_char_p, [P]),
@@ -198,7 +199,7 @@ class Hyat:
                                   s.cuda_stream), self.handle)
         return out
 
-    def stream_step(self, q, k, v, mask=None, out=None, stream=None):
+    def _stream_call(self, fn, q, k, v, mask, out, stream):
         c = self.cfg
         L = c.chunk_frames * c.tokens_per_frame
         for t, nm in ((q, "q"), (k, "k"), (v, "v")):
@@ -207,9 +208,18 @@ class Hyat:
         self._check_t(out, "out", L)
         m = None if mask is None else _u8(mask)
         s = torch.cuda.current_stream(q.device) if stream is None else stream
-        _check(lib.hyat_fwd_stream_step(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                        None if m is None else m.ctypes.data, s.cuda_stream), self.handle)
+        _check(fn(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                  None if m is None else m.ctypes.data, s.cuda_stream), self.handle)
         return out
+
+    def stream_step(self, q, k, v, mask=None, out=None, stream=None):
+        """The current chunk's final call: attend, then keep its K, V and advance."""
+        return self._stream_call(lib.hyat_fwd_stream_step, q, k, v, mask, out, stream)
+
+    def stream_denoise(self, q, k, v, mask=None, out=None, stream=None):
+        """A non-final call for the current chunk (one denoising step): attend with this
+        call's K, V as the newest chunk, without advancing."""
+        return self._stream_call(lib.hyat_fwd_stream_denoise, q, k, v, mask, out, stream)
 
     def sync(self):
         _check(lib.hyat_sync(self.handle), self.handle)

@@ -21,7 +21,8 @@ Random draw recipe (all configs):
   * cast to the workload dtype with round-to-nearest-even (torch ``.to``).
 Streaming steps use ``default_rng([seed, step])`` and draw Q, K, V of the
 current chunk, then the block mask (``random(...) < 0.5``), then force the
-diagonal tiles on.
+diagonal tiles on. A chunk's earlier denoising calls draw the same way from
+``default_rng([seed, step, 1000 + call])``.
 """
 from __future__ import annotations
 
@@ -123,14 +124,18 @@ def stream_window_chunks(w: Workload, step: int) -> int:
     return min(step + 1, w.window_frames // w.chunk_frames)
 
 
-def gen_stream_step(w: Workload, step: int, seed: Optional[int] = None, keep_prob: float = 0.5):
+def gen_stream_step(w: Workload, step: int, seed: Optional[int] = None, keep_prob: float = 0.5,
+                    call: Optional[int] = None):
     """Q, K, V of chunk ``step`` ([B,H,chunk_tokens,d]) and its tile mask.
 
     The mask is uint8 [H, tiles_per_chunk, tiles_per_chunk * n_window_chunks];
     key tiles are ordered oldest window chunk first. Tile (i, j) of the newest
     chunk's diagonal is always set; the rest is Bernoulli(keep_prob).
+    ``call`` selects the inputs of an earlier (non-final) denoising call of the
+    chunk, drawn from their own stream; None gives the chunk's final inputs.
     """
-    rng = np.random.default_rng([w.seed if seed is None else seed, step])
+    base = [w.seed if seed is None else seed, step]
+    rng = np.random.default_rng(base if call is None else base + [1000 + call])
     shape = (w.B, w.H, w.chunk_tokens, w.d)
     q = rng.standard_normal(shape, dtype=np.float32)
     k = rng.standard_normal(shape, dtype=np.float32)

@@ -103,10 +103,13 @@ def test_radial_small(T, F):
 
 
 # ------------------------------------------------------------------ streaming
+STATE_HEADER_BYTES = 48   # magic, version, step, BH, d, L, nwc, dtype, folded step, 3 reserved
+
+
 def _state_from_blob(blob, BH, d):
-    hdr = np.frombuffer(blob[:32], np.int32)
+    hdr = np.frombuffer(blob[:STATE_HEADER_BYTES], np.int32)
     E = d * d + d
-    s = np.frombuffer(blob[32:32 + 4 * BH * E], np.float32).reshape(BH, E)
+    s = np.frombuffer(blob[STATE_HEADER_BYTES:STATE_HEADER_BYTES + 4 * BH * E], np.float32).reshape(BH, E)
     return int(hdr[2]), s[:, :d * d].reshape(BH, d, d), s[:, d * d:]
 
 
@@ -189,6 +192,73 @@ def test_stream_checkpoint_resume_bit_identical():
         q, k, v, mask = wl.gen_stream_step(w, s)
         o = h2.stream_step(*_dev(q, k, v), mask=mask).cpu()
         assert torch.equal(o, ref_outs[s]), s
+    h2.close()
+
+
+def test_stream_denoise_calls_then_final_call():
+    """Several denoising calls per chunk, then the final call: every call attends to the
+    committed window, the folded state and its own K, V; only the final K, V stay."""
+    w = wl.Workload("stream_denoise", "stream", 1, 2, 128, 200, 24, chunk_frames=3, window_frames=9,
+                    n_steps=6, seed=5)
+    h = hyat.Hyat(hyat.config_from_workload(w, mask_heads=2))
+    L, nwc = w.chunk_tokens, w.window_frames // w.chunk_frames
+    kh, vh = [], []
+    for s in range(6):
+        for call in range(2):
+            q, k, v, mask = wl.gen_stream_step(w, s, call=call)
+            o = h.stream_denoise(*_dev(q, k, v), mask=mask)
+            h.sync()
+            k_all = np.concatenate(kh + [k.float().numpy()], axis=2)
+            v_all = np.concatenate(vh + [v.float().numpy()], axis=2)
+            ref = oracle.stream_step_attention(f64(q), k_all, v_all, s, L, nwc, mask)
+            assert_parity("bf16", f64(o), ref, f"chunk {s} denoising call {call}")
+        q, k, v, mask = wl.gen_stream_step(w, s)
+        o = h.stream_step(*_dev(q, k, v), mask=mask)
+        h.sync()
+        kh.append(k.float().numpy())
+        vh.append(v.float().numpy())
+        ref = oracle.stream_step_attention(f64(q), np.concatenate(kh, axis=2), np.concatenate(vh, axis=2),
+                                           s, L, nwc, mask)
+        assert_parity("bf16", f64(o), ref, f"chunk {s} final call")
+    step, S, z = _state_from_blob(h.get_state(), 2, 128)
+    assert step == 6
+    # the folded state holds the final K, V of chunks 0..2 only; the bound is the one of
+    # test_stream_small_steps_and_state (bf16 phi(k) operand, fp32 accumulation)
+    k_all, v_all = np.concatenate(kh, axis=2), np.concatenate(vh, axis=2)
+    S_ref, z_ref = oracle.stream_evicted_state(k_all, v_all, 5, L, 3)
+    n_ev = 3 * L
+    pk = oracle.phi_elu1(k_all[:, :, :n_ev])
+    bound_S = 2.0 ** -8 * np.einsum("bhna,bhnc->bhac", pk, np.abs(v_all[:, :, :n_ev]))
+    bound_z = 2.0 ** -8 * pk.sum(axis=2)
+    assert np.all(np.abs(S.reshape(1, 2, 128, 128) - S_ref) <= bound_S + 1e-5 * np.abs(S_ref).max())
+    assert np.all(np.abs(z.reshape(1, 2, 128) - z_ref) <= bound_z + 1e-5 * np.abs(z_ref).max())
+    h.close()
+
+
+def test_stream_checkpoint_between_denoising_calls_bit_identical():
+    """A state saved after a chunk's denoising call (its fold done) resumes exactly."""
+    w = wl.Workload("stream_ckpt_mid", "stream", 1, 2, 128, 200, 24, chunk_frames=3, window_frames=9,
+                    n_steps=6, seed=9)
+    cfg = hyat.config_from_workload(w, mask_heads=2)
+    h1 = hyat.Hyat(cfg)
+    for s in range(4):
+        h1.stream_step(*_dev(*wl.gen_stream_step(w, s)[:3]), mask=wl.gen_stream_step(w, s)[3])
+    q, k, v, mask = wl.gen_stream_step(w, 4, call=0)
+    h1.stream_denoise(*_dev(q, k, v), mask=mask)        # chunk 4: folds chunk 1
+    h1.sync()
+    blob = h1.get_state()
+    seq = [("denoise", wl.gen_stream_step(w, 4, call=1)), ("step", wl.gen_stream_step(w, 4)),
+           ("step", wl.gen_stream_step(w, 5))]
+    ref = []
+    for kind, (q, k, v, mask) in seq:
+        fn = h1.stream_denoise if kind == "denoise" else h1.stream_step
+        ref.append(fn(*_dev(q, k, v), mask=mask).cpu())
+    h1.close()
+    h2 = hyat.Hyat(cfg)
+    h2.set_state(blob)
+    for (kind, (q, k, v, mask)), r in zip(seq, ref):
+        fn = h2.stream_denoise if kind == "denoise" else h2.stream_step
+        assert torch.equal(fn(*_dev(q, k, v), mask=mask).cpu(), r), kind
     h2.close()
 
 
