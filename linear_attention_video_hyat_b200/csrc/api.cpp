@@ -315,9 +315,14 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   if (e == cudaSuccess && !h->lay.entries.empty())
     e = cudaMemcpy(h->d_entries, h->lay.entries.data(), sizeof(Entry) * h->lay.entries.size(),
                    cudaMemcpyHostToDevice);
-  const std::vector<int4> pairs = cfg->mode == HYAT_MODE_STREAM
-                                      ? build_stream_pairs(h->BH, tiles(stream_chunk_tokens(*cfg)))
-                                      : order_pairs_for_grid(build_pairs(h->lay.work), h->lay.work, h->num_sms);
+  std::vector<int4> pairs;
+  if (cfg->mode == HYAT_MODE_STREAM) {
+    const int32_t nqt = tiles(stream_chunk_tokens(*cfg));
+    pairs = build_stream_pairs(h->BH, nqt);
+    if (prefer_split_pairs(pairs.size(), h->num_sms)) pairs = build_split_pairs(size_t(h->BH) * nqt);
+  } else {
+    pairs = choose_pairs(h->lay.work, h->num_sms);
+  }
   h->n_pairs = static_cast<int32_t>(pairs.size());
   if (e == cudaSuccess && !pairs.empty())
     e = cudaMemcpy(h->d_pairs, pairs.data(), sizeof(int4) * pairs.size(), cudaMemcpyHostToDevice);

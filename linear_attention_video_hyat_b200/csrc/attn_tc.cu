@@ -65,7 +65,9 @@ struct __align__(1024) Smem {
   uint64_t kv_full[NS], kv_empty[NS];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t xfull, o1_free;       // split pairs: slot 1's (l, m) handed over; O1 read out
   uint64_t drain;
+  float2 xchg[128];              // split pairs: slot 1's (l, m) per row
   uint32_t tmem_base;
   int32_t abort_flag;
   uint64_t never;                // test hook: a barrier nothing arrives on
@@ -75,7 +77,7 @@ struct __align__(1024) Smem {
 struct TcParams {
   const WorkItem* work;
   const Entry* entries;
-  const int4* pairs;       // {item0, item1 (-1 = none), shared key list, 0}
+  const int4* pairs;       // {item0, item1 (-1 = none), shared key list, split}
   int32_t n_pairs;
   const float* srest;      // [groups][d*d + d] fp32; z at offset d*d
   void* o;
@@ -137,6 +139,47 @@ __device__ __forceinline__ float exp_tile(const uint32_t (&r)[128], float sl, fl
   return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
+// What each slot does for a pair. A split pair {item, item, 0, 1} runs one query tile on both
+// slots: slot 0 takes the first half of its key tiles (and the linear term), slot 1 the
+// second half, and slot 0's warpgroup merges the two partial results. Split pairs keep a
+// grid of few query tiles busy (a streaming chunk of 37 tiles per head gives 1.5 waves of
+// ordinary pairs on 148 SMs, and 3 waves of split pairs).
+struct PairView {
+  int item[2];
+  int eb[2];            // first entry of each slot's key tiles
+  int n[2];             // number of key tiles of each slot
+  bool has1, shared, split;
+};
+
+__device__ __forceinline__ PairView pair_view(const TcParams& p, int pi) {
+  const int4 pr = p.pairs[pi];
+  PairView v;
+  const WorkItem w0 = p.work[pr.x];
+  const int n = w0.entry_end - w0.entry_begin;
+  v.item[0] = pr.x;
+  v.eb[0] = w0.entry_begin;
+  if (pr.w != 0) {
+    const int n0 = (n + 1) / 2;
+    v.item[1] = pr.x;
+    v.eb[1] = w0.entry_begin + n0;
+    v.n[0] = n0;
+    v.n[1] = n - n0;
+    v.has1 = n - n0 > 0;
+    v.split = v.has1;
+    v.shared = false;
+  } else {
+    v.item[1] = pr.y;
+    v.has1 = pr.y >= 0;
+    const WorkItem w1 = v.has1 ? p.work[pr.y] : w0;
+    v.eb[1] = w1.entry_begin;
+    v.n[0] = n;
+    v.n[1] = v.has1 ? w1.entry_end - w1.entry_begin : 0;
+    v.split = false;
+    v.shared = pr.z != 0;
+  }
+  return v;
+}
+
 // One query row per thread (TMEM lane = row). Slot s = warpgroup index.
 __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32_t tmem, int warp) {
   const int s = warp >> 2;
@@ -149,26 +192,34 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
   uint64_t* p_full = &sm->p_full[s];
   uint64_t* pv_done = &sm->pv_done[s];
   const float sl = p.scale_log2;
-  uint32_t qph = 0, sph = 0;
+  uint32_t qph = 0, sph = 0, xph = 0;
   uint32_t pv_phase = 0;                            // pv_done phases completed before this pair
+  bool o1_busy = false;                             // slot 1: O1 not yet read out by slot 0
   for (int pi = blockIdx.x; pi < p.n_pairs; pi += gridDim.x) {
-    const int4 pr = p.pairs[pi];
-    const int item = s == 0 ? pr.x : pr.y;
-    if (item < 0) continue;
-    const WorkItem wi = p.work[item];
-    const int n = wi.entry_end - wi.entry_begin;
-    const Entry* ent = p.entries + wi.entry_begin;
+    const PairView pv = pair_view(p, pi);
+    if (s == 1 && !pv.has1) continue;
+    const WorkItem wi = p.work[s == 0 ? pv.item[0] : pv.item[1]];
+    const int n = s == 0 ? pv.n[0] : pv.n[1];
+    const Entry* ent = p.entries + (s == 0 ? pv.eb[0] : pv.eb[1]);
+    // slot 1 of a split pair carries no linear term and starts O1 with its first P.V
+    const bool lin = !(pv.split && s == 1);
     int klen_next = n > 0 ? ent[0].k_len : 128;
     if (!wait_warp(q_full, qph, sm, p.status)) return;
     qph ^= 1u;
-    // phi(q) of this row -> TMEM (bf16 pairs), l = phi(q) . z
-    // z_rest of this tile's group: each lane holds 4 values (one coalesced 512-byte load per
-    // warp) and the phi loop broadcasts them with shuffles
-    const float4 zq = __ldg(reinterpret_cast<const float4*>(
-        p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D) + (row & 31));
-    const float zreg[4] = {zq.x, zq.y, zq.z, zq.w};
+    if (o1_busy) {
+      // O1 is rewritten once this warpgroup hands over its next operand: wait until slot 0
+      // has read out the previous split pair's O1
+      if (!wait_warp(&sm->o1_free, xph ^ 1u, sm, p.status)) return;
+      o1_busy = false;
+    }
     float l = 0.0f, m = 0.0f;
-    {
+    if (lin) {
+      // phi(q) of this row -> TMEM (bf16 pairs), l = phi(q) . z
+      // z_rest of this tile's group: each lane holds 4 values (one coalesced 512-byte load per
+      // warp) and the phi loop broadcasts them with shuffles
+      const float4 zq = __ldg(reinterpret_cast<const float4*>(
+          p.srest + (static_cast<int64_t>(wi.bh) * p.nqg + wi.state_group) * (D * D + D) + D * D) + (row & 31));
+      const float zreg[4] = {zq.x, zq.y, zq.z, zq.w};
       const uint8_t* qrow = sm->q[s] + row * 128;
       float lz[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
@@ -227,7 +278,11 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
         const float mrow = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
         const float m_new = fmaxf(m, mrow * sl);
         const float alpha = ex2(m - m_new);
-        if (!wait_warp(pv_done, (pv_phase + j) & 1u, sm, p.status)) return;
+        // Rescale O once its last product so far (commit j - 1 + lin of this pair) has
+        // landed. On slot 1 of a split pair at j = 0 nothing has been committed yet: the wait
+        // is for the previous pair's last phase (already complete), and the values scaled
+        // are overwritten by the first P.V, which starts the accumulator.
+        if (!wait_warp(pv_done, (pv_phase + j - 1 + (lin ? 1u : 0u)) & 1u, sm, p.status)) return;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -248,32 +303,62 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    // epilogue: o = O / l, bf16, 16-byte stores of the valid rows
-    if (!wait_warp(pv_done, (pv_phase + n) & 1u, sm, p.status)) return;
-    pv_phase += n + 1;
+    const uint32_t n_commits = static_cast<uint32_t>(n) + (lin ? 1u : 0u);
+    if (!wait_warp(pv_done, (pv_phase + n_commits - 1) & 1u, sm, p.status)) return;
+    pv_phase += n_commits;
     tc_fence_after();
-    const float inv = 1.0f / l;
+    if (pv.split && s == 1) {
+      // hand (l, m) and O1 to slot 0's warpgroup, which merges and stores the tile
+      sm->xchg[row] = make_float2(l, m);
+      tc_fence_before();
+      mbar_arrive(&sm->xfull);
+      xph ^= 1u;
+      o1_busy = true;
+      continue;
+    }
+    // epilogue: o = O / l (merged with slot 1's half for split pairs), bf16, 16-byte stores
+    float a0 = 1.0f, a1 = 0.0f, inv;
+    if (pv.split) {
+      if (!wait_warp(&sm->xfull, xph, sm, p.status)) return;
+      xph ^= 1u;
+      tc_fence_after();
+      const float2 o1s = sm->xchg[row];
+      const float mm = fmaxf(m, o1s.y);
+      a0 = ex2(m - mm);
+      a1 = ex2(o1s.y - mm);
+      inv = 1.0f / (l * a0 + o1s.x * a1);
+    } else {
+      inv = 1.0f / l;
+    }
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
                                           (static_cast<int64_t>(wi.bh) * p.q_rows + wi.q_row + row) * D);
 #pragma unroll 1
-    for (int h = 0; h < 2; ++h) {
-      uint32_t r[64];
-      tmem_ld32p(tO + h * 64, r);
-      tmem_ld32p(tO + h * 64 + 32, r + 32);
-      tmem_wait_ld();
+    for (int h = 0; h < 4; ++h) {               // 32 columns at a time
+      uint32_t r[32];
+      tmem_ld32p(tO + h * 32, r);
+      if (pv.split) {
+        uint32_t r1[32];
+        tmem_ld32p(tO + 128 + h * 32, r1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(fmaf(u2f(r[i]), a0, u2f(r1[i]) * a1));
+      } else {
+        tmem_wait_ld();
+      }
       if (row < wi.q_len) {
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
+        for (int v = 0; v < 4; ++v) {
           uint4 w;
           w.x = pack_bf16(u2f(r[8 * v + 0]) * inv, u2f(r[8 * v + 1]) * inv);
           w.y = pack_bf16(u2f(r[8 * v + 2]) * inv, u2f(r[8 * v + 3]) * inv);
           w.z = pack_bf16(u2f(r[8 * v + 4]) * inv, u2f(r[8 * v + 5]) * inv);
           w.w = pack_bf16(u2f(r[8 * v + 6]) * inv, u2f(r[8 * v + 7]) * inv);
-          dst[h * 8 + v] = w;
+          dst[h * 4 + v] = w;
         }
       }
     }
     tc_fence_before();
+    if (pv.split) mbar_arrive(&sm->o1_free);
   }
 }
 
@@ -298,6 +383,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&sm->p_full[s], 128);
       mbar_init(&sm->pv_done[s], 1);
     }
+    mbar_init(&sm->xfull, 128);
+    mbar_init(&sm->o1_free, 128);
     mbar_init(&sm->drain, 1);
     mbar_init(&sm->never, 1);
     sm->abort_flag = 0;
@@ -333,15 +420,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return true;
       };
       for (int pi = blockIdx.x; pi < p.n_pairs && ok; pi += gridDim.x) {
-        const int4 pr = p.pairs[pi];
-        const bool has1 = pr.y >= 0, shared = pr.z != 0;
-        const WorkItem w0 = p.work[pr.x];
-        WorkItem w1 = w0;
-        if (has1) w1 = p.work[pr.y];
-        const int n0 = w0.entry_end - w0.entry_begin;
-        const int n1 = has1 ? w1.entry_end - w1.entry_begin : 0;
-        const Entry* e0 = p.entries + w0.entry_begin;
-        const Entry* e1 = p.entries + w1.entry_begin;
+        const PairView pv = pair_view(p, pi);
+        const bool has1 = pv.has1, shared = pv.shared;
+        const WorkItem w0 = p.work[pv.item[0]];
+        const WorkItem w1 = has1 ? p.work[pv.item[1]] : w0;
+        const int n0 = pv.n[0], n1 = pv.n[1];
+        const Entry* e0 = p.entries + pv.eb[0];
+        const Entry* e1 = p.entries + pv.eb[1];
         ok = mbar_wait(&sm->q_empty[0], qph0 ^ 1u, sm, p.status);
         if (!ok) break;
         qph0 ^= 1u;
@@ -355,7 +440,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = take(&tmS, 0, w0.bh * p.nqg + w0.state_group);
         if (ok && n0 > 0) ok = take(&tmK, e0[0].k_row, w0.bh);
         if (ok && has1) {
-          ok = take(&tmS, 0, w1.bh * p.nqg + w1.state_group);
+          if (!pv.split) ok = take(&tmS, 0, w1.bh * p.nqg + w1.state_group);   // no linear term on split slot 1
           if (ok && n1 > 0 && !shared) ok = take(&tmK, e1[0].k_row, w1.bh);
         }
         const int nmax = n0 > n1 ? n0 : n1;
@@ -411,10 +496,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < 8; ++kk) mma_ss_elect(tS, dq + koff(kk), dk + koff(kk), kIdescKK, kk > 0);
         mma_commit_elect(done);
       };
-      auto pv = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
+      // first = true starts the accumulator (slot 1 of a split pair has no linear term)
+      auto pv = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done, bool first) {
         const uint64_t dv = dV0 + static_cast<uint64_t>(stage) * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_ts_elect(tO, tS + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescKMN, 1);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts_elect(tO, tS + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), kIdescKMN, (first && kk == 0) ? 0 : 1);
         mma_commit_elect(done);
       };
       auto linear = [&](uint32_t tO, uint32_t tS, int stage, uint64_t* done) {
@@ -425,10 +512,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
       for (int pi = blockIdx.x; pi < p.n_pairs && ok; pi += gridDim.x) {
-        const int4 pr = p.pairs[pi];
-        const bool has1 = pr.y >= 0, shared = pr.z != 0;
-        const int n0 = p.work[pr.x].entry_end - p.work[pr.x].entry_begin;
-        const int n1 = has1 ? p.work[pr.y].entry_end - p.work[pr.y].entry_begin : 0;
+        const PairView pvw = pair_view(p, pi);
+        const bool has1 = pvw.has1, shared = pvw.shared, split = pvw.split;
+        const int n0 = pvw.n[0], n1 = pvw.n[1];
         int k0 = -1, k1 = -1, v0 = -1, v1 = -1, sst = -1;
         // slot 0: O0 = phi(Q0) S_rest (S_rest [a][b] is the MN-major B operand), then S0 = Q0 K^T
         ok = wait_p(&sm->p_full[0], pph0) && next_stage(sst);
@@ -448,10 +534,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (n0 <= 1) mma_commit_elect(&sm->q_empty[0]);
         // slot 1
         if (has1) {
-          ok = wait_p(&sm->p_full[1], pph1) && next_stage(sst);
-          if (!ok) break;
-          linear(tO1, tS1, sst, &sm->pv_done[1]);
-          mma_commit_elect(&sm->kv_empty[sst]);
+          if (!split) {
+            ok = wait_p(&sm->p_full[1], pph1) && next_stage(sst);
+            if (!ok) break;
+            linear(tO1, tS1, sst, &sm->pv_done[1]);
+            mma_commit_elect(&sm->kv_empty[sst]);
+          }
           ok = mbar_wait_warp(&sm->q_full[1], qph1, sm, p.status);
           if (!ok) break;
           qph1 ^= 1u;
@@ -472,7 +560,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!(ok = next_stage(v0))) break;
             if (j + 1 < n0 && !(ok = next_stage(k0))) break;
             if (!(ok = wait_p(&sm->p_full[0], pph0))) break;
-            pv(tO0, tS0, v0, &sm->pv_done[0]);
+            pv(tO0, tS0, v0, &sm->pv_done[0], false);
             if (!shared) mma_commit_elect(&sm->kv_empty[v0]);
             if (j + 1 < n0) {
               qk(tS0, dQ0, k0, &sm->s_full[0]);
@@ -489,7 +577,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if (j + 1 < n1 && !(ok = next_stage(k1))) break;
             }
             if (!(ok = wait_p(&sm->p_full[1], pph1))) break;
-            pv(tO1, tS1, v1, &sm->pv_done[1]);
+            pv(tO1, tS1, v1, &sm->pv_done[1], split && j == 0);
             mma_commit_elect(&sm->kv_empty[v1]);
             if (j + 1 < n1) {
               qk(tS1, dQ1, k1, &sm->s_full[1]);
@@ -522,6 +610,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ------------------------------------------------------------------ host side
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB a CTA can have");
 
 }  // namespace
 

@@ -59,6 +59,13 @@ std::vector<int4> build_pairs(const std::vector<WorkItem>& work);
 std::vector<int4> order_pairs_for_grid(const std::vector<int4>& pairs, const std::vector<WorkItem>& work,
                                        int32_t grid);
 std::vector<int4> build_stream_pairs(int32_t BH, int32_t nqt);
+// One split pair {i, i, 0, 1} per work item: both slots of a CTA run the same query tile,
+// each over half of its key tiles, and the halves are merged in the epilogue.
+std::vector<int4> build_split_pairs(size_t n_items);
+// Split pairs when ordinary pairs would give the persistent grid fewer than four waves.
+bool prefer_split_pairs(size_t n_ordinary_pairs, int32_t num_sms);
+// build_pairs or build_split_pairs (by prefer_split_pairs), then order_pairs_for_grid.
+std::vector<int4> choose_pairs(const std::vector<WorkItem>& work, int32_t num_sms);
 void radial_tile_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t* out);
 
 // ---- kernel launch wrappers (kernels_simt.cu, attn_tc.cu) ----

@@ -235,6 +235,22 @@ std::vector<int4> order_pairs_for_grid(const std::vector<int4>& pairs, const std
   return out;
 }
 
+std::vector<int4> build_split_pairs(size_t n_items) {
+  std::vector<int4> pairs(n_items);
+  for (size_t i = 0; i < n_items; ++i) pairs[i] = make_int4(static_cast<int>(i), static_cast<int>(i), 0, 1);
+  return pairs;
+}
+
+bool prefer_split_pairs(size_t n_ordinary_pairs, int32_t num_sms) {
+  return n_ordinary_pairs < static_cast<size_t>(4) * static_cast<size_t>(num_sms > 0 ? num_sms : 1);
+}
+
+std::vector<int4> choose_pairs(const std::vector<WorkItem>& work, int32_t num_sms) {
+  std::vector<int4> pairs = build_pairs(work);
+  if (prefer_split_pairs(pairs.size(), num_sms)) pairs = build_split_pairs(work.size());
+  return order_pairs_for_grid(pairs, work, num_sms);
+}
+
 std::vector<int4> build_stream_pairs(int32_t BH, int32_t nqt) {
   std::vector<int4> pairs;
   for (int32_t bh = 0; bh < BH; ++bh)

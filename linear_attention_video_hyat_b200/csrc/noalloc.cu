@@ -70,7 +70,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
 
   Layout L;
   if (!build_layout(*cfg, nullptr, &L).empty()) return HYAT_ERR_INVALID_ARG;
-  std::vector<int4> pairs = build_pairs(L.work);
+  std::vector<int4> pairs;   // chosen once the SM count is known; at most one per work item
   const int64_t BH = int64_t(cfg->B) * cfg->H;
   const int64_t E = int64_t(cfg->d) * cfg->d + cfg->d;
   const int64_t rows = rows_q(*cfg);
@@ -81,7 +81,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   const size_t o_status = take(256);
   const size_t o_work = take(sizeof(WorkItem) * L.work.size());
   const size_t o_entries = take(sizeof(Entry) * (L.entries.empty() ? 1 : L.entries.size()));
-  const size_t o_pairs = take(sizeof(int4) * pairs.size());
+  const size_t o_pairs = take(sizeof(int4) * (L.work.empty() ? 1 : L.work.size()));
   const size_t o_cm = take(sizeof(float) * L.cm.size());
   const size_t o_sseg = take(sizeof(float) * size_t(BH) * L.nseg * E);
   const size_t o_srest = take(sizeof(float) * size_t(BH) * L.nqg * E);
@@ -91,7 +91,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   void* base = nullptr;
   int num_sms = 0;
   if (scratch_for_current_device(&base, &num_sms) != cudaSuccess) return HYAT_ERR_CUDA;
-  pairs = order_pairs_for_grid(pairs, L.work, num_sms);
+  pairs = choose_pairs(L.work, num_sms);
   char* ws = static_cast<char*>(base);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 

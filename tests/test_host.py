@@ -4,6 +4,7 @@ import os
 import re
 
 import numpy as np
+import torch
 import pytest
 
 import oracle
@@ -131,3 +132,21 @@ def test_workspace_sizes():
     for w in (wl.TINY_F32, wl.WAN13B_BIDIR, wl.WAN14B_BIDIR, wl.STREAM_HF, wl.RADIAL_84F):
         n = hyat.workspace_bytes(hyat.config_from_workload(w))
         assert 0 < n < 4 << 30, (w.name, n)
+
+
+def test_peaked_bf16_bound_accepts_rounding_and_rejects_a_planted_error():
+    """The large-logit tolerance admits bf16 rounding of o and P, and no more."""
+    import pytest as _pt
+    from parity import assert_bf16_peaked
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal((1, 1, 64, 16))
+    s = 40.0 * rng.standard_normal((1, 1, 8, 64))           # nearly one-hot softmax rows
+    p = np.exp(s - s.max(axis=3, keepdims=True))
+    ref = (p @ v[0, 0]) / p.sum(axis=3, keepdims=True)
+    bf = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).double().numpy()
+    o = bf((bf(p) @ v[0, 0]) / p.sum(axis=3, keepdims=True))  # P and o rounded to bf16
+    assert_bf16_peaked(o, ref, v)
+    bad = o.copy()
+    bad[0, 0, 3, 5] += 2.0 ** -8 * (abs(ref[0, 0, 3, 5]) + np.abs(v).max()) * 1.5
+    with _pt.raises(AssertionError):
+        assert_bf16_peaked(bad, ref, v)
