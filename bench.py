@@ -198,6 +198,167 @@ def cpu_rate(w, counts, n_blocks, qkv=None):
     return tflops, rows / secs, secs, rows
 
 
+# ----------------------------------------------------------------- streaming workload
+def stream_step_flops(w, mask, fold):
+    """Effective FLOPs of one streaming step: 4d per (query, key) pair inside kept tiles, the
+    fold of one evicted chunk (if any) and the linear term applied to every query."""
+    L, d, BH = w.chunk_tokens, w.d, w.B * w.H
+    nqt = wl.stream_tiles_per_chunk(w)
+    qlen = np.minimum(wl.TILE, L - wl.TILE * np.arange(nqt)).astype(np.int64)
+    klen = np.tile(qlen, mask.shape[2] // nqt)
+    per_head = np.einsum("hij,i,j->h", mask.astype(np.int64), qlen, klen)
+    pairs = int(per_head.sum()) * (w.B * w.H // mask.shape[0])
+    soft = 4 * d * pairs
+    apply = BH * L * (2 * d * d + 2 * d)
+    folded = BH * L * (2 * d * d + d) if fold else 0
+    return soft + apply + folded, soft + apply
+
+
+def bench_stream(a, w, rank, world, local):
+    """Streaming steps of chunk `w.chunk_tokens` tokens: K steady steps after W warm-up steps."""
+    from linear_attention_video_hyat_b200 import hyat
+    nwc = w.window_frames // w.chunk_frames
+    warm = max(a.warmup, nwc, 3)
+    config = {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "chunk_tokens": w.chunk_tokens,
+              "tokens_per_frame": w.tokens_per_frame, "chunk_frames": w.chunk_frames,
+              "window_frames": w.window_frames, "mode": w.mode, "mask": "Bernoulli(0.5) + diagonal tiles",
+              "parallelism": f"replicas{world}" if world > 1 else "single",
+              "l2": "per step: fresh Q, K, V (86 MB) and the ring (86 MB); no flush"}
+    n_dist = 4           # distinct steady-state inputs, cycled
+    inputs = [wl.gen_stream_step(w, nwc + i, seed=w.seed + rank) for i in range(n_dist)]
+    flops = [stream_step_flops(w, m, True) for _, _, _, m in inputs]
+    mean_flops = float(np.mean([f[0] for f in flops]))
+    mean_attn = float(np.mean([f[1] for f in flops]))
+    if a.impl == "reference":
+        if rank != 0:
+            return 0
+        import oracle
+        L = w.chunk_tokens
+        hist = [wl.gen_stream_step(w, s, seed=w.seed) for s in range(nwc + 1)]
+        kh = np.concatenate([x[1].float().numpy() for x in hist], axis=2)
+        vh = np.concatenate([x[2].float().numpy() for x in hist], axis=2)
+        q, mask = hist[-1][0].float().numpy(), hist[-1][3]
+        rng = np.random.default_rng(0)
+        secs, rows_done = 0.0, 0
+        for i in range(a.warmup + a.steps):
+            hh = int(rng.integers(0, w.H))
+            r0 = int(rng.integers(0, L - 256 + 1))
+            t0 = time.perf_counter()
+            oracle.stream_step_attention(q[:, hh:hh + 1], kh[:, hh:hh + 1], vh[:, hh:hh + 1], nwc, L, nwc,
+                                         mask[hh:hh + 1], rows=np.arange(r0, r0 + 256))
+            if i >= a.warmup:
+                secs += time.perf_counter() - t0
+                rows_done += 256
+        frac = rows_done / (w.B * w.H * L)
+        value = mean_flops * frac / secs / 1e12
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus, "steps": a.steps,
+                "warmup": a.warmup, "ms_per_step": 1e3 * secs / a.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "impl": "reference", "tokens_per_s": rows_done / secs,
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                                 "sample": f"{a.steps} blocks of 256 query rows (one head each) of a steady step"},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    cfg = hyat.config_from_workload(w, mask_heads=w.H)
+    dev_in = [(q.to(dev), k.to(dev), v.to(dev), m) for q, k, v, m in inputs]
+    od = torch.empty_like(dev_in[0][0])
+    stream = torch.cuda.current_stream(dev)
+
+    def run(h, steps, first):
+        for i in range(steps):
+            s = first + i
+            q, k, v, m = dev_in[s % n_dist]
+            if s < nwc:       # the window is still filling: masks of the growing shape
+                m = wl.gen_stream_step(w, s, seed=w.seed + rank)[3]
+            h.stream_step(q, k, v, mask=m, out=od)
+
+    h = hyat.Hyat(cfg, device=dev)
+    run(h, warm, 0)
+    h.sync()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        run(h, a.steps, warm)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    h.sync()
+    ms = max_over_ranks(t0.elapsed_time(t1) / a.steps, dev)
+    h.set_profiling(True)
+    h.kernel_times()
+    with ClockSampler(local) as clk2:
+        run(h, a.steps, warm + a.steps)
+        torch.cuda.synchronize(dev)
+    kt = h.kernel_times()
+    h.set_profiling(False)
+    launches = sum(n for _, n in kt.values())
+    value, tokens_per_s = job_throughput(mean_flops, w.B * w.chunk_tokens, ms, world)
+    pk, pk_src = peaks()
+    attn_ms = kt["attention"][0] / max(kt["attention"][1], 1)
+    achieved = mean_attn / (attn_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attention", "achieved": achieved,
+                "timing": "per-launch CUDA events over a second pass of K steps",
+                "clocks_kernel_pass": clk2.summary(), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"], "peak_kind": f"{pk_src} bf16 burst",
+                "peak_sustained": pk["bf16_tflops_sustained"],
+                "frac_sustained": achieved / pk["bf16_tflops_sustained"], "traffic": None,
+                "launch_ms": attn_ms, "algorithmic_flops_per_launch": mean_attn}
+    kernels = {k_: {"ms_per_launch": t_ / max(n_, 1), "launches": n_} for k_, (t_, n_) in kt.items() if n_}
+
+    e2e = None
+    if not a.no_e2e:
+        pinned = [tuple(t.pin_memory() for t in x[:3]) + (x[3],) for x in inputs]
+        oh = torch.empty_like(pinned[0][0]).pin_memory()
+        qd, kd, vd = (torch.empty_like(t) for t in dev_in[0][:3])
+        e_steps = max(3, min(a.steps, 20))
+
+        def run_e2e(first, steps):
+            for i in range(steps):
+                qh, kh_, vh, m = pinned[(first + i) % n_dist]
+                qd.copy_(qh, non_blocking=True); kd.copy_(kh_, non_blocking=True); vd.copy_(vh, non_blocking=True)
+                h.stream_step(qd, kd, vd, mask=m, out=od)
+                oh.copy_(od, non_blocking=True)
+        run_e2e(0, 2)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run_e2e(2, e_steps)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = max_over_ranks(e0.elapsed_time(e1) / e_steps, dev)
+        e_value, e_tokens = job_throughput(mean_flops, w.B * w.chunk_tokens, ems, world)
+        q0 = inputs[0][0]
+        e2e = {"value": e_value, "unit": "TFLOP/s", "ms_per_step": ems, "tokens_per_s": e_tokens,
+               "h2d_bytes_per_step": 3 * q0.numel() * q0.element_size() + int(inputs[0][3].nbytes),
+               "d2h_bytes_per_step": q0.numel() * q0.element_size()}
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+                "warmup": warm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+                "tokens_per_s": tokens_per_s, "frac_of_peak": value / world / pk["bf16_tflops"],
+                "effective_flops_per_step": mean_flops * world, "roofline": roofline, "kernels": kernels,
+                "gpu_launches": launches, "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": None}
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------- main
 def main():
     a = parse()
@@ -205,7 +366,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
     w = wl.WORKLOADS[a.workload]
-    assert w.mode in ("window", "radial"), "the bench times a bidirectional layer call"
+    if w.mode == "stream":
+        return bench_stream(a, w, rank, world, local)
+    assert w.mode in ("window", "radial"), "the bench times a bidirectional layer call or streaming steps"
     counts = work_counts(w)
     config = {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "tokens": w.N,
               "tokens_per_frame": w.tokens_per_frame, "frames": w.n_frames, "mode": w.mode,

@@ -13,7 +13,8 @@
  *
  *   o_i = ( sum_{j in W_i} e^{s_ij - m_i} v_j + e^{-m_i} phi(q_i)^T S )
  *       / ( sum_{j in W_i} e^{s_ij - m_i}     + e^{-m_i} phi(q_i)^T z ),
- *   s_ij = scale * q_i . k_j,   phi(x) = elu(x) + 1,   m_i = max(0, max_j s_ij).
+ *   s_ij = scale * q_i . k_j,   phi(x) = elu(x) + 1 (or ReLU, exp: hyat_phi),
+ *   m_i = max(0, max_j s_ij).
  *
  * Modes (hyat_config.mode):
  *   WINDOW     bidirectional; frames of tokens_per_frame tokens are grouped in
@@ -76,7 +77,10 @@ typedef enum {
 } hyat_status;
 
 typedef enum { HYAT_F32 = 0, HYAT_BF16 = 1 } hyat_dtype;
-typedef enum { HYAT_PHI_ELU1 = 0 } hyat_phi;
+/* Feature map of the linear branch. The pages leave it open (the hybrid normaliser
+ * needs phi >= 0); elu + 1 is the default. ReLU and exp are the other maps of the
+ * linear-attention literature the pages cite (Transformers are RNNs; Hedgehog). */
+typedef enum { HYAT_PHI_ELU1 = 0, HYAT_PHI_RELU = 1, HYAT_PHI_EXP = 2 } hyat_phi;
 typedef enum {
   HYAT_MODE_WINDOW = 0,
   HYAT_MODE_BLOCKMASK = 1,

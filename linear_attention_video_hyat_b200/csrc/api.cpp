@@ -202,6 +202,7 @@ AttnArgs attn_args(hyat_ctx* h, const void* q, const void* k, const void* v, voi
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = h->d_status;
   a.test_timeout = (h->cfg.flags & HYAT_FLAG_TEST_DEVICE_TIMEOUT) ? 1 : 0;
+  a.phi = h->cfg.phi;
   return a;
 }
 
@@ -372,7 +373,7 @@ hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const vo
   const Layout& L = h->lay;
   SegStateArgs sa{};
   sa.k = k; sa.v = v; sa.rows_per_bh = h->rk;
-  sa.BH = h->BH; sa.d = h->cfg.d; sa.dtype = h->cfg.dtype;
+  sa.BH = h->BH; sa.d = h->cfg.d; sa.dtype = h->cfg.dtype; sa.phi = h->cfg.phi;
   sa.nseg = L.nseg; sa.seg_base = 0; sa.seg_stride = L.seg_stride; sa.seg_len = L.seg_len;
   sa.out = h->d_sseg; sa.accumulate = 0; sa.status = h->d_status;
   if (h->use_gemm) {        // hi/lo bf16 parts for the tensor-core complement, in the same bytes
@@ -446,7 +447,7 @@ hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void*
     if (fold) {  // chunk s - nwc leaves the window: fold it into S, z
       SegStateArgs sa{};
       sa.k = h->d_ring_k; sa.v = h->d_ring_v; sa.rows_per_bh = h->rk;
-      sa.BH = h->BH; sa.d = c.d; sa.dtype = c.dtype;
+      sa.BH = h->BH; sa.d = c.d; sa.dtype = c.dtype; sa.phi = c.phi;
       sa.nseg = 1; sa.seg_base = slot * Lc; sa.seg_stride = Lc; sa.seg_len = Lc;
       sa.out = h->d_srest; sa.accumulate = 1; sa.status = h->d_status;
       if (h->use_tc) {

@@ -86,6 +86,7 @@ struct TcParams {
   float scale_log2;
   uint32_t* status;
   int32_t test_timeout;    // test hook: wait once on a barrier nothing signals (20 ms limit)
+  int32_t phi;             // feature map of the linear branch (hyat_phi)
 };
 
 // Bounded wait on a phase parity. Returns false if the kernel is aborting. After the first
@@ -233,7 +234,7 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-          const float f0 = phi_elu1(f.x), f1 = phi_elu1(f.y);
+          const float f0 = phi_map(f.x, p.phi), f1 = phi_map(f.y, p.phi);
           lz[e] = fmaf(f0, zz[2 * e], lz[e]);
           lz[e] = fmaf(f1, zz[2 * e + 1], lz[e]);
           pk[e] = pack_bf16(f0, f1);
@@ -642,6 +643,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s) {
   p.scale_log2 = a.scale_log2;
   p.status = a.status;
   p.test_timeout = a.test_timeout;
+  p.phi = a.phi;
   const int grid = a.n_pairs < num_sms ? a.n_pairs : num_sms;
   return launch_pdl(attn_tc_kernel, dim3(grid), dim3(NUM_THREADS), kSmemBytes, s, mq, mk, mv, ms, p);
 }

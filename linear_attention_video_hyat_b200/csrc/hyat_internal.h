@@ -84,6 +84,7 @@ struct SegStateArgs {
   int32_t parts;
   int32_t part_len;
   float* partial;
+  int32_t phi;                // hyat_phi
 };
 cudaError_t launch_seg_state(const SegStateArgs& a, cudaStream_t s);
 
@@ -140,6 +141,7 @@ struct AttnArgs {
   float scale_log2;           // scale * log2(e)
   uint32_t* status;
   int32_t test_timeout;       // HYAT_FLAG_TEST_DEVICE_TIMEOUT (tensor-core path)
+  int32_t phi;                // hyat_phi
 };
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s);

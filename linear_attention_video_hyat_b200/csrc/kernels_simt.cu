@@ -20,7 +20,12 @@ template <> __device__ __forceinline__ float from_f<float>(float x) { return x; 
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 // phi(x) = elu(x) + 1 with alpha = 1
-__device__ __forceinline__ float phi_elu1(float x) { return x > 0.0f ? x + 1.0f : expf(x); }
+// Feature maps of the linear branch (hyat_phi): 0 elu + 1, 1 ReLU, 2 exp.
+__device__ __forceinline__ float phi_map(float x, int kind) {
+  if (kind == 1) return fmaxf(x, 0.0f);
+  if (kind == 2) return expf(x);
+  return x > 0.0f ? x + 1.0f : expf(x);
+}
 
 // four consecutive elements as floats (p must be 8-byte (bf16) / 16-byte (f32) aligned)
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
@@ -60,7 +65,7 @@ __global__ void __launch_bounds__(256) seg_state_kernel(SegStateArgs a) {
       float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), vv = kk;
       if (t0 + r < len) {
         kk = ld4(K + static_cast<int64_t>(t0 + r) * D + 64 * at + c4);
-        kk = make_float4(phi_elu1(kk.x), phi_elu1(kk.y), phi_elu1(kk.z), phi_elu1(kk.w));
+        kk = make_float4(phi_map(kk.x, a.phi), phi_map(kk.y, a.phi), phi_map(kk.z, a.phi), phi_map(kk.w, a.phi));
         vv = ld4(V + static_cast<int64_t>(t0 + r) * D + 64 * bt + c4);
       }
       *reinterpret_cast<float4*>(&Ks[r][c4]) = kk;
@@ -295,7 +300,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
     __syncthreads();
     for (int r = 0; r < BK; ++r) {
       const float4 qv = *reinterpret_cast<const float4*>(&Qs[(a0 + r) * PQ + 4 * ty]);
-      const float pq[4] = {phi_elu1(qv.x), phi_elu1(qv.y), phi_elu1(qv.z), phi_elu1(qv.w)};
+      const float pq[4] = {phi_map(qv.x, a.phi), phi_map(qv.y, a.phi), phi_map(qv.z, a.phi), phi_map(qv.w, a.phi)};
 #pragma unroll
       for (int u = 0; u < NU; ++u) {
         const float4 sv = *reinterpret_cast<const float4*>(&Vs[r * PD + 4 * tx + 64 * u]);
@@ -314,10 +319,10 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
       const int c = tx * PER + r;
       const float4 qv = *reinterpret_cast<const float4*>(&Qs[c * PQ + 4 * ty]);
       const float zc = z[c];
-      l[0] = fmaf(phi_elu1(qv.x), zc, l[0]);
-      l[1] = fmaf(phi_elu1(qv.y), zc, l[1]);
-      l[2] = fmaf(phi_elu1(qv.z), zc, l[2]);
-      l[3] = fmaf(phi_elu1(qv.w), zc, l[3]);
+      l[0] = fmaf(phi_map(qv.x, a.phi), zc, l[0]);
+      l[1] = fmaf(phi_map(qv.y, a.phi), zc, l[1]);
+      l[2] = fmaf(phi_map(qv.z, a.phi), zc, l[2]);
+      l[3] = fmaf(phi_map(qv.w, a.phi), zc, l[3]);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)

@@ -35,7 +35,8 @@ std::string validate_config(const hyat_config& c) {
   if (c.d != 64 && c.d != 128) return "d must be 64 or 128";
   if (c.tokens_per_frame < 1) return "tokens_per_frame must be >= 1";
   if (c.dtype != HYAT_F32 && c.dtype != HYAT_BF16) return "dtype must be HYAT_F32 or HYAT_BF16";
-  if (c.phi != HYAT_PHI_ELU1) return "phi must be HYAT_PHI_ELU1";
+  if (c.phi != HYAT_PHI_ELU1 && c.phi != HYAT_PHI_RELU && c.phi != HYAT_PHI_EXP)
+    return "phi must be HYAT_PHI_ELU1, HYAT_PHI_RELU or HYAT_PHI_EXP";
   if (!(c.scale >= 0.0f) || std::isinf(c.scale)) return "scale must be finite and >= 0";
   switch (c.mode) {
     case HYAT_MODE_WINDOW:

@@ -109,7 +109,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
 
   SegStateArgs sa{};
   sa.k = k; sa.v = v; sa.rows_per_bh = rows;
-  sa.BH = static_cast<int32_t>(BH); sa.d = cfg->d; sa.dtype = cfg->dtype;
+  sa.BH = static_cast<int32_t>(BH); sa.d = cfg->d; sa.dtype = cfg->dtype; sa.phi = cfg->phi;
   sa.nseg = L.nseg; sa.seg_base = 0; sa.seg_stride = L.seg_stride; sa.seg_len = L.seg_len;
   sa.out = reinterpret_cast<float*>(ws + o_sseg); sa.accumulate = 0;
   if (launch_seg_state(sa, s) != cudaSuccess) return HYAT_ERR_CUDA;
@@ -144,6 +144,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   const float scale = cfg->scale > 0.0f ? cfg->scale : 1.0f / sqrtf(float(cfg->d));
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = reinterpret_cast<uint32_t*>(ws + o_status);
+  a.phi = cfg->phi;
 
   if (use_tc) {
     if (launch_attn_tc(a, num_sms, s) != cudaSuccess) return HYAT_ERR_CUDA;

@@ -60,6 +60,7 @@ struct StateParams {
   uint32_t* status;
   uint16_t* out_hi;          // if set: bf16 hi/lo parts instead of fp32 `out`
   uint16_t* out_lo;
+  int32_t phi;               // feature map (hyat_phi)
 };
 
 __device__ __forceinline__ bool swait(uint64_t* b, uint32_t parity, StateSmem* sm, uint32_t* status) {
@@ -103,6 +104,118 @@ __device__ __forceinline__ Unit unit_of(const StateParams& p, int u) {
   x.len = static_cast<int>(rem < len ? (rem > 0 ? rem : 0) : len);
   x.ntiles = x.len > 0 ? (x.len + TOK - 1) / TOK : 1;
   return x;
+}
+
+// Warps 0-3: apply phi in place to the K half of each stage (rows past the unit's end become
+// zero), then hand the stage to the MMA warp.
+template <int kKind>
+__device__ __forceinline__ void phi_role(StateSmem* sm, const StateParams& p) {
+  // phi in place: thread t owns column chunk t % 16 of rows t / 16 + 8 k
+  const int t = threadIdx.x;
+  const int cc = t & 15, half = cc >> 3, c8 = cc & 7;
+  int st = 0;
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    const Unit x = unit_of(p, u);
+    for (int i = 0; i < x.ntiles; ++i) {
+      if (!(ok = swait_warp(&sm->full[st], ph, sm, p.status))) break;
+      const int valid = x.len - TOK * i;
+      uint8_t* kt = sm->stage[st] + half * KT_HALF;
+#pragma unroll 4
+      for (int k = 0; k < TOK / 8; ++k) {
+        const int r = (t >> 4) + 8 * k;
+        uint4* addr = reinterpret_cast<uint4*>(kt + r * 128 + ((c8 ^ (r & 7)) << 4));
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (r < valid) {
+          const uint4 raw = *addr;
+          const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t o4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
+            o4[e] = pack_bf16(phi_of<kKind>(f.x), phi_of<kKind>(f.y));
+          }
+          w = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+        *addr = w;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&sm->phi_done[st]);
+      if (++st == NST) { st = 0; ph ^= 1u; }
+    }
+  }
+}
+
+// Warps 4-7: drain a finished accumulator (S_g and z_g) to global memory while the next unit
+// accumulates in the other TMEM buffer.
+__device__ __forceinline__ void drain_role(StateSmem* sm, const StateParams& p, uint32_t tmem, int warp, int lane) {
+  // drain: row a of S_g (TMEM lane a) and z_g[a]
+  const int a = (warp & 3) * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  int c = 0;
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++c) {
+    const Unit x = unit_of(p, u);
+    const int buf = c & 1;
+    if (!swait_warp(&sm->acc_full[buf], (c >> 1) & 1, sm, p.status)) break;
+    tc_fence_after();
+    const uint32_t tacc = tmem + buf * 256 + lane_off;
+    const int64_t obase = (static_cast<int64_t>(x.bh) * p.nseg + x.g) * (D * D + D);
+    float* out = p.partial ? p.partial + static_cast<int64_t>(u) * (D * D + D) : p.out + obase;
+    const bool acc_out = p.accumulate && !p.partial;
+    uint32_t zr[1];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(zr[0]) : "r"(tacc + 128));
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      uint32_t r[64];
+      tmem_ld32p(tacc + 64 * h, r);
+      tmem_ld32p(tacc + 64 * h + 32, r + 32);
+      tmem_wait_ld();
+      if (h == 1) {
+        tc_fence_before();
+        mbar_arrive(&sm->acc_empty[buf]);
+      }
+      if (p.out_hi) {
+        // hi = bf16(x), lo = bf16(x - hi): 16-byte stores of 8 values each
+        uint4* dhi = reinterpret_cast<uint4*>(p.out_hi + obase + a * D + 64 * h);
+        uint4* dlo = reinterpret_cast<uint4*>(p.out_lo + obase + a * D + 64 * h);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float x0 = u2f(r[8 * v + 2 * t]), x1 = u2f(r[8 * v + 2 * t + 1]);
+            hw[t] = pack_bf16(x0, x1);
+            const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[t]));
+            lw[t] = pack_bf16(x0 - hf.x, x1 - hf.y);
+          }
+          dhi[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          dlo[v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(out + a * D + 64 * h);
+#pragma unroll
+        for (int v = 0; v < 16; ++v) {
+          float4 val = make_float4(u2f(r[4 * v]), u2f(r[4 * v + 1]), u2f(r[4 * v + 2]), u2f(r[4 * v + 3]));
+          if (acc_out) {
+            const float4 o = dst[v];
+            val.x += o.x; val.y += o.y; val.z += o.z; val.w += o.w;
+          }
+          dst[v] = val;
+        }
+      }
+    }
+    const float zv = u2f(zr[0]);
+    if (p.out_hi) {
+      const __nv_bfloat16 zh = __float2bfloat16_rn(zv);
+      const __nv_bfloat16 zl = __float2bfloat16_rn(zv - __bfloat162float(zh));
+      p.out_hi[obase + D * D + a] = *reinterpret_cast<const uint16_t*>(&zh);
+      p.out_lo[obase + D * D + a] = *reinterpret_cast<const uint16_t*>(&zl);
+    } else {
+      float* zp = out + D * D + a;
+      *zp = acc_out ? *zp + zv : zv;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(ST_THREADS, 1)
@@ -208,108 +321,11 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
       }
     }
   } else if (warp < 4) {
-    // phi in place: thread t owns column chunk t % 16 of rows t / 16 + 8 k
-    const int t = threadIdx.x;
-    const int cc = t & 15, half = cc >> 3, c8 = cc & 7;
-    int st = 0;
-    uint32_t ph = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit x = unit_of(p, u);
-      for (int i = 0; i < x.ntiles; ++i) {
-        if (!(ok = swait_warp(&sm->full[st], ph, sm, p.status))) break;
-        const int valid = x.len - TOK * i;
-        uint8_t* kt = sm->stage[st] + half * KT_HALF;
-#pragma unroll 4
-        for (int k = 0; k < TOK / 8; ++k) {
-          const int r = (t >> 4) + 8 * k;
-          uint4* addr = reinterpret_cast<uint4*>(kt + r * 128 + ((c8 ^ (r & 7)) << 4));
-          uint4 w = make_uint4(0u, 0u, 0u, 0u);
-          if (r < valid) {
-            const uint4 raw = *addr;
-            const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
-            uint32_t o4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
-              o4[e] = pack_bf16(phi_elu1(f.x), phi_elu1(f.y));
-            }
-            w = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-          }
-          *addr = w;
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive(&sm->phi_done[st]);
-        if (++st == NST) { st = 0; ph ^= 1u; }
-      }
-    }
+    if (p.phi == 1) phi_role<1>(sm, p);
+    else if (p.phi == 2) phi_role<2>(sm, p);
+    else phi_role<0>(sm, p);
   } else {
-    // drain: row a of S_g (TMEM lane a) and z_g[a]
-    const int a = (warp & 3) * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    int c = 0;
-    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++c) {
-      const Unit x = unit_of(p, u);
-      const int buf = c & 1;
-      if (!swait_warp(&sm->acc_full[buf], (c >> 1) & 1, sm, p.status)) break;
-      tc_fence_after();
-      const uint32_t tacc = tmem + buf * 256 + lane_off;
-      const int64_t obase = (static_cast<int64_t>(x.bh) * p.nseg + x.g) * (D * D + D);
-      float* out = p.partial ? p.partial + static_cast<int64_t>(u) * (D * D + D) : p.out + obase;
-      const bool acc_out = p.accumulate && !p.partial;
-      uint32_t zr[1];
-      asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(zr[0]) : "r"(tacc + 128));
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        uint32_t r[64];
-        tmem_ld32p(tacc + 64 * h, r);
-        tmem_ld32p(tacc + 64 * h + 32, r + 32);
-        tmem_wait_ld();
-        if (h == 1) {
-          tc_fence_before();
-          mbar_arrive(&sm->acc_empty[buf]);
-        }
-        if (p.out_hi) {
-          // hi = bf16(x), lo = bf16(x - hi): 16-byte stores of 8 values each
-          uint4* dhi = reinterpret_cast<uint4*>(p.out_hi + obase + a * D + 64 * h);
-          uint4* dlo = reinterpret_cast<uint4*>(p.out_lo + obase + a * D + 64 * h);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const float x0 = u2f(r[8 * v + 2 * t]), x1 = u2f(r[8 * v + 2 * t + 1]);
-              hw[t] = pack_bf16(x0, x1);
-              const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[t]));
-              lw[t] = pack_bf16(x0 - hf.x, x1 - hf.y);
-            }
-            dhi[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            dlo[v] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(out + a * D + 64 * h);
-#pragma unroll
-          for (int v = 0; v < 16; ++v) {
-            float4 val = make_float4(u2f(r[4 * v]), u2f(r[4 * v + 1]), u2f(r[4 * v + 2]), u2f(r[4 * v + 3]));
-            if (acc_out) {
-              const float4 o = dst[v];
-              val.x += o.x; val.y += o.y; val.z += o.z; val.w += o.w;
-            }
-            dst[v] = val;
-          }
-        }
-      }
-      const float zv = u2f(zr[0]);
-      if (p.out_hi) {
-        const __nv_bfloat16 zh = __float2bfloat16_rn(zv);
-        const __nv_bfloat16 zl = __float2bfloat16_rn(zv - __bfloat162float(zh));
-        p.out_hi[obase + D * D + a] = *reinterpret_cast<const uint16_t*>(&zh);
-        p.out_lo[obase + D * D + a] = *reinterpret_cast<const uint16_t*>(&zl);
-      } else {
-        float* zp = out + D * D + a;
-        *zp = acc_out ? *zp + zv : zv;
-      }
-    }
+    drain_role(sm, p, tmem, warp, lane);
   }
 
   tc_fence_before();
@@ -319,7 +335,6 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
 }
-
 constexpr size_t kStateSmemBytes = sizeof(StateSmem) + 1024;
 
 }  // namespace
@@ -355,6 +370,7 @@ cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t
   p.status = a.status;
   p.out_hi = a.out_hi;
   p.out_lo = a.out_lo;
+  p.phi = a.phi;
   const int grid = p.n_units < num_sms ? p.n_units : num_sms;
   state_tc_kernel<<<grid, ST_THREADS, kStateSmemBytes, s>>>(mk, mv, p);
   return cudaGetLastError();

@@ -202,8 +202,15 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 
-__device__ __forceinline__ float phi_elu1(float x) {
+// Feature maps of the linear branch (hyat_phi): 0 elu + 1, 1 ReLU, 2 exp.
+template <int kKind>
+__device__ __forceinline__ float phi_of(float x) {
+  if (kKind == 1) return fmaxf(x, 0.0f);
+  if (kKind == 2) return ex2(x * 1.4426950408889634f);
   return x > 0.0f ? x + 1.0f : ex2(x * 1.4426950408889634f);
+}
+__device__ __forceinline__ float phi_map(float x, int kind) {
+  return kind == 1 ? phi_of<1>(x) : kind == 2 ? phi_of<2>(x) : phi_of<0>(x);
 }
 
 

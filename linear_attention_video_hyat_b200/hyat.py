@@ -89,17 +89,22 @@ def _load():
 lib = _load()
 
 
+PHI = {"elu1": 0, "relu": 1, "exp": 2}   # hyat_phi
+
+
 def make_config(mode, B, H, d, tokens_per_frame, n_frames=0, chunk_frames=1, halo_frames=0,
-                window_frames=0, dtype=BF16, mask_heads=1, flags=0, scale=0.0) -> Config:
+                window_frames=0, dtype=BF16, mask_heads=1, flags=0, scale=0.0, phi="elu1") -> Config:
     m = _MODES[mode] if isinstance(mode, str) else int(mode)
     dt = {"f32": F32, "bf16": BF16}.get(dtype, dtype) if isinstance(dtype, str) else int(dtype)
+    ph = PHI[phi] if isinstance(phi, str) else int(phi)
     return Config(B, H, d, tokens_per_frame, n_frames, chunk_frames, halo_frames, window_frames,
-                  m, dt, 0, mask_heads, flags, float(scale))
+                  m, dt, ph, mask_heads, flags, float(scale))
 
 
 def config_from_workload(w, flags=0, mask_heads=1) -> Config:
     return make_config(w.mode, w.B, w.H, w.d, w.tokens_per_frame, w.n_frames, w.chunk_frames,
-                       w.halo_frames, w.window_frames, w.dtype, mask_heads=mask_heads, flags=flags)
+                       w.halo_frames, w.window_frames, w.dtype, mask_heads=mask_heads, flags=flags,
+                       phi=getattr(w, "phi", "elu1"))
 
 
 def _check(status, handle=None):

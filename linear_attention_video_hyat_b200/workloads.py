@@ -51,6 +51,7 @@ class Workload:
     dtype: str = "bf16"        # "f32" | "bf16"
     per_head_std: bool = False
     seed: int = 0
+    phi: str = "elu1"          # feature map of the linear branch: "elu1" | "relu" | "exp"
     note: str = ""
 
     @property

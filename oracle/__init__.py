@@ -10,6 +10,10 @@ brute force, invariants); none is "parity unpinned".
 """
 from .hybrid import (  # noqa: F401
     phi_elu1,
+    phi_relu,
+    phi_exp,
+    FEATURE_MAPS,
+    feature_map,
     hybrid_rows,
     bidir_window_interval,
     bidir_sets,

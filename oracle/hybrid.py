@@ -24,8 +24,8 @@ Here m_i = max(0, max_{j in W_i} s_ij) only keeps exp() in range.
 
 Readings taken where the pages are silent (each is listed with its reason in
 the design notes):
-  * phi = elu + 1 with alpha = 1, on raw q and k; the scale multiplies softmax
-    logits only.
+  * phi = elu + 1 with alpha = 1 by default (ReLU and exp on request), on raw q
+    and k; the scale multiplies softmax logits only.
   * bidirectional window: chunk c covers frames [c*C, (c+1)*C); its window is
     frames [c*C - halo, (c+1)*C + halo) clipped to the video.
   * radial mask: tile kept iff any token pair in it is "near"; near means same
@@ -51,10 +51,31 @@ def phi_elu1(x):
     return np.where(x > 0.0, x + 1.0, np.exp(np.minimum(x, 0.0)))
 
 
+def phi_relu(x):
+    """phi(x) = max(x, 0)."""
+    return np.maximum(np.asarray(x, dtype=np.float64), 0.0)
+
+
+def phi_exp(x):
+    """phi(x) = exp(x), elementwise."""
+    return np.exp(np.asarray(x, dtype=np.float64))
+
+
+# The pages leave the feature map open (only phi >= 0 is needed for one normaliser);
+# elu + 1 is the default, ReLU and exp are the alternatives of the linear-attention papers
+# the pages cite.
+FEATURE_MAPS = {"elu1": phi_elu1, "relu": phi_relu, "exp": phi_exp}
+
+
+def feature_map(phi):
+    """A feature map given by name ("elu1", "relu", "exp") or as a function."""
+    return FEATURE_MAPS[phi] if isinstance(phi, str) else phi
+
+
 # --------------------------------------------------------------------------
 # the definition, for a block of rows
 # --------------------------------------------------------------------------
-def hybrid_rows(q_rows, k, v, soft, lin, scale):
+def hybrid_rows(q_rows, k, v, soft, lin, scale, phi=phi_elu1):
     """Outputs of the rows in ``q_rows`` [R,d] against keys k [N,d], values v [N,d].
 
     ``soft`` and ``lin`` are disjoint boolean masks [R,N]: the softmax set and
@@ -70,7 +91,7 @@ def hybrid_rows(q_rows, k, v, soft, lin, scale):
     s_win = np.where(soft, s, -np.inf)
     m = np.maximum(0.0, np.max(s_win, axis=1, initial=-np.inf))
     e_soft = np.exp(s_win - m[:, None])                 # 0 outside the window
-    lin_w = (phi_elu1(q_rows) @ phi_elu1(k).T) * np.exp(-m)[:, None]
+    lin_w = (phi(q_rows) @ phi(k).T) * np.exp(-m)[:, None]
     e_lin = np.where(lin, lin_w, 0.0)
     num_soft = e_soft @ v
     den_soft = e_soft.sum(axis=1)
@@ -80,7 +101,7 @@ def hybrid_rows(q_rows, k, v, soft, lin, scale):
     return o, num_soft, den_soft, num_lin, den_lin
 
 
-def _run_rows(q, k, v, rows, sets_fn, scale, with_branches=False):
+def _run_rows(q, k, v, rows, sets_fn, scale, with_branches=False, phi="elu1"):
     """Apply hybrid_rows per (batch, head) over the requested rows.
 
     q: [B,H,Nq,d]; k, v: [B,H,Nk,d]; sets_fn(h, rows) -> (soft, lin).
@@ -100,7 +121,7 @@ def _run_rows(q, k, v, rows, sets_fn, scale, with_branches=False):
                 rr = rows[r0:r0 + ROW_BLOCK]
                 soft, lin = sets_fn(h, rr)
                 qb = np.asarray(q[b, h, rr], dtype=np.float64)
-                o, ns, ds, nl, dl = hybrid_rows(qb, kb, vb, soft, lin, scale)
+                o, ns, ds, nl, dl = hybrid_rows(qb, kb, vb, soft, lin, scale, feature_map(phi))
                 out[b, h, r0:r0 + len(rr)] = o
                 if with_branches:
                     br[0][b, h, r0:r0 + len(rr)] = ns
@@ -143,11 +164,11 @@ def bidir_sets(rows, tokens_per_frame, n_frames, chunk_frames, halo_frames):
 
 
 def bidir_window_attention(q, k, v, tokens_per_frame, n_frames, chunk_frames,
-                           halo_frames, scale=None, rows=None, with_branches=False):
+                           halo_frames, scale=None, rows=None, with_branches=False, phi="elu1"):
     """Bidirectional hybrid attention: window = chunk +/- halo frames, the rest linear."""
     sc = _default_scale(q.shape[-1], scale)
     fn = lambda h, rr: bidir_sets(rr, tokens_per_frame, n_frames, chunk_frames, halo_frames)
-    return _run_rows(q, k, v, rows, fn, sc, with_branches)
+    return _run_rows(q, k, v, rows, fn, sc, with_branches, phi)
 
 
 # --------------------------------------------------------------------------
@@ -167,11 +188,11 @@ def tile_mask_sets(h, rows, tile_mask, N, tile=128):
 
 
 def blockmask_attention(q, k, v, tile_mask, scale=None, rows=None, tile=128,
-                        with_branches=False):
+                        with_branches=False, phi="elu1"):
     N = q.shape[2]
     sc = _default_scale(q.shape[-1], scale)
     fn = lambda h, rr: tile_mask_sets(h, rr, tile_mask, N, tile)
-    return _run_rows(q, k, v, rows, fn, sc, with_branches)
+    return _run_rows(q, k, v, rows, fn, sc, with_branches, phi)
 
 
 # --------------------------------------------------------------------------
@@ -239,9 +260,9 @@ def radial_tile_mask(n_frames, tokens_per_frame, tile=128):
 
 
 def radial_attention(q, k, v, n_frames, tokens_per_frame, scale=None, rows=None,
-                     tile=128, with_branches=False):
+                     tile=128, with_branches=False, phi="elu1"):
     mask = radial_tile_mask(n_frames, tokens_per_frame, tile)[None]
-    return blockmask_attention(q, k, v, mask, scale, rows, tile, with_branches)
+    return blockmask_attention(q, k, v, mask, scale, rows, tile, with_branches, phi)
 
 
 # --------------------------------------------------------------------------
@@ -271,15 +292,15 @@ def stream_sets(h, rows, step, chunk_tokens, n_window_chunks, tile_mask, tile=12
 
 
 def stream_step_attention(q_chunk, k_hist, v_hist, step, chunk_tokens, n_window_chunks,
-                          tile_mask, scale=None, rows=None, tile=128, with_branches=False):
+                          tile_mask, scale=None, rows=None, tile=128, with_branches=False, phi="elu1"):
     """Output of chunk ``step``; k_hist, v_hist hold chunks 0..step ([B,H,(step+1)L,d])."""
     assert k_hist.shape[2] == (step + 1) * chunk_tokens
     sc = _default_scale(q_chunk.shape[-1], scale)
     fn = lambda h, rr: stream_sets(h, rr, step, chunk_tokens, n_window_chunks, tile_mask, tile)
-    return _run_rows(q_chunk, k_hist, v_hist, rows, fn, sc, with_branches)
+    return _run_rows(q_chunk, k_hist, v_hist, rows, fn, sc, with_branches, phi)
 
 
-def stream_evicted_state(k_hist, v_hist, step, chunk_tokens, n_window_chunks):
+def stream_evicted_state(k_hist, v_hist, step, chunk_tokens, n_window_chunks, phi="elu1"):
     """Linear state used at ``step``: S = sum phi(k) v^T, z = sum phi(k) over evicted chunks.
 
     Returns S [B,H,d,d] and z [B,H,d] in float64 (zero before anything is evicted).
@@ -287,7 +308,7 @@ def stream_evicted_state(k_hist, v_hist, step, chunk_tokens, n_window_chunks):
     n_evicted = max(0, step - n_window_chunks + 1) * chunk_tokens
     k = np.asarray(k_hist[:, :, :n_evicted], dtype=np.float64)
     v = np.asarray(v_hist[:, :, :n_evicted], dtype=np.float64)
-    pk = phi_elu1(k)
+    pk = feature_map(phi)(k)
     S = np.einsum("bhna,bhnc->bhac", pk, v)
     z = pk.sum(axis=2)
     return S, z

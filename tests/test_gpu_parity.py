@@ -262,6 +262,50 @@ def test_stream_checkpoint_between_denoising_calls_bit_identical():
     h2.close()
 
 
+# ------------------------------------------------------------------ feature maps
+@pytest.mark.parametrize("phi", ["relu", "exp"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_feature_map_window(phi, dtype):
+    w = wl.Workload("phi_window", "window", 1, 2, 128, 300, 6, 2, 1, dtype=dtype, seed=23, phi=phi)
+    o, (q, k, v) = _bidir(w)
+    ref = oracle.bidir_window_attention(f64(q), f64(k), f64(v), w.tokens_per_frame, w.n_frames,
+                                        w.chunk_frames, w.halo_frames, phi=phi)
+    assert_parity(dtype, f64(o), ref, (phi, dtype))
+
+
+@pytest.mark.parametrize("phi", ["relu", "exp"])
+def test_feature_map_blockmask(phi):
+    """Diagonal tile mask with query tile 0 left empty (pure linear attention for its rows)."""
+    T, F, H = 4, 230, 2
+    nT = -(-T * F // 128)
+    mask = np.zeros((H, nT, nT), np.uint8)
+    mask[:, np.arange(nT), np.arange(nT)] = 1
+    mask[:, 0, :] = 0
+    w = wl.Workload("phi_bm", "blockmask", 1, H, 128, F, T, seed=29, phi=phi)
+    o, (q, k, v) = _bidir(w, mask=mask, mask_heads=H)
+    ref = oracle.blockmask_attention(f64(q), f64(k), f64(v), mask, phi=phi)
+    assert_parity("bf16", f64(o), ref, phi)
+
+
+@pytest.mark.parametrize("phi", ["relu", "exp"])
+def test_feature_map_stream(phi):
+    w = wl.Workload("phi_stream", "stream", 1, 2, 128, 200, 18, chunk_frames=3, window_frames=9,
+                    n_steps=6, seed=31, phi=phi)
+    h = hyat.Hyat(hyat.config_from_workload(w, mask_heads=2))
+    L, nwc = w.chunk_tokens, w.window_frames // w.chunk_frames
+    kh, vh = [], []
+    for s in range(6):
+        q, k, v, mask = wl.gen_stream_step(w, s)
+        o = h.stream_step(*_dev(q, k, v), mask=mask)
+        h.sync()
+        kh.append(k.float().numpy())
+        vh.append(v.float().numpy())
+        ref = oracle.stream_step_attention(f64(q), np.concatenate(kh, axis=2), np.concatenate(vh, axis=2),
+                                           s, L, nwc, mask, phi=phi)
+        assert_parity("bf16", f64(o), ref, (phi, s))
+    h.close()
+
+
 # ------------------------------------------------------------------ errors
 def test_invalid_calls_return_errors_and_handle_stays_usable():
     w = wl.Workload("err", "stream", 1, 2, 64, 100, 9, chunk_frames=3, window_frames=6, n_steps=2, seed=1)

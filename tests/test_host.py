@@ -117,7 +117,7 @@ def test_stream_plan_eviction_indexing():
 
 @pytest.mark.parametrize("bad", [dict(d=96), dict(B=0), dict(tokens_per_frame=0), dict(mode=9),
                                  dict(mode="stream", window_frames=8), dict(mode="blockmask", mask_heads=3),
-                                 dict(dtype=7), dict(scale=-1.0)])
+                                 dict(dtype=7), dict(scale=-1.0), dict(phi=3), dict(phi=-1)])
 def test_invalid_configs_rejected(bad):
     kw = dict(mode="window", B=1, H=2, d=64, tokens_per_frame=64, n_frames=4, chunk_frames=1,
               window_frames=9)
@@ -150,3 +150,9 @@ def test_peaked_bf16_bound_accepts_rounding_and_rejects_a_planted_error():
     bad[0, 0, 3, 5] += 2.0 ** -8 * (abs(ref[0, 0, 3, 5]) + np.abs(v).max()) * 1.5
     with _pt.raises(AssertionError):
         assert_bf16_peaked(bad, ref, v)
+
+
+@pytest.mark.parametrize("phi", ["elu1", "relu", "exp"])
+def test_feature_maps_accepted(phi):
+    cfg = hyat.make_config("window", 1, 2, 64, 64, 4, 1, 0, phi=phi)
+    assert hyat.workspace_bytes(cfg) > 0

@@ -33,6 +33,19 @@ def test_phi_is_elu_plus_one():
     assert np.all(oracle.phi_elu1(x) > 0)
 
 
+def test_phi_relu_and_exp_closed_forms():
+    x = np.concatenate([_rand(2000, 2, 3.0), [0.0, -0.0, 1e-300, -1e-300, -40.0, 40.0]])
+    # ReLU: (x + |x|) / 2, zero exactly on x <= 0
+    np.testing.assert_array_equal(oracle.phi_relu(x), (x + np.abs(x)) / 2)
+    assert np.all(oracle.phi_relu(x[x <= 0]) == 0.0)
+    # exp: exp(0) = 1, exp(ln 2) = 2, and exp(a) exp(b) = exp(a + b)
+    assert oracle.phi_exp(0.0) == 1.0
+    np.testing.assert_allclose(oracle.phi_exp(np.log(2.0)), 2.0, rtol=1e-15)
+    a, b = _rand(500, 3), _rand(500, 4)
+    np.testing.assert_allclose(oracle.phi_exp(a) * oracle.phi_exp(b), oracle.phi_exp(a + b), rtol=1e-14)
+    assert oracle.feature_map("elu1") is oracle.phi_elu1 and set(oracle.FEATURE_MAPS) == {"elu1", "relu", "exp"}
+
+
 # ------------------------------------------------------------------- limits
 def test_window_all_is_softmax_attention():
     """One chunk spanning the whole video: the linear set is empty."""
@@ -48,13 +61,17 @@ def test_window_all_is_softmax_attention():
     np.testing.assert_allclose(o2, ref, rtol=1e-11, atol=1e-13)
 
 
-def test_empty_window_is_linear_attention():
+_TORCH_PHI = {"elu1": lambda t: torch.nn.functional.elu(t) + 1, "relu": torch.relu, "exp": torch.exp}
+
+
+@pytest.mark.parametrize("phi", ["elu1", "relu", "exp"])
+def test_empty_window_is_linear_attention(phi):
     """An all-zero tile mask: every key reaches the query through phi(q).phi(k)."""
     B, H, N, d = 1, 3, 80, 16
     q, k, v = (_rand((B, H, N, d), s) for s in (4, 5, 6))
-    o = oracle.blockmask_attention(q, k, v, np.zeros((H, 10, 10), np.uint8), tile=8)
-    pq = torch.nn.functional.elu(torch.from_numpy(q)).numpy() + 1
-    pk = torch.nn.functional.elu(torch.from_numpy(k)).numpy() + 1
+    o = oracle.blockmask_attention(q, k, v, np.zeros((H, 10, 10), np.uint8), tile=8, phi=phi)
+    pq = _TORCH_PHI[phi](torch.from_numpy(q)).numpy()
+    pk = _TORCH_PHI[phi](torch.from_numpy(k)).numpy()
     S = np.einsum("bhna,bhnc->bhac", pk, v)          # associativity: (phi K)^T V first
     z = pk.sum(axis=2)
     ref = np.einsum("bhna,bhac->bhnc", pq, S) / np.einsum("bhna,bha->bhn", pq, z)[..., None]
@@ -62,7 +79,15 @@ def test_empty_window_is_linear_attention():
 
 
 # -------------------------------------------------------------- brute force
-def _bruteforce(q, k, v, in_soft, in_lin, scale):
+def _phi_scalar(x, phi):
+    if phi == "relu":
+        return x if x > 0 else 0.0
+    if phi == "exp":
+        return float(np.e) ** x
+    return x + 1 if x > 0 else np.exp(x)
+
+
+def _bruteforce(q, k, v, in_soft, in_lin, scale, phi="elu1"):
     """Explicit N x N weight matrix with plain loops, no stabiliser."""
     n, d = q.shape
     out = np.zeros((n, v.shape[1]))
@@ -75,9 +100,7 @@ def _bruteforce(q, k, v, in_soft, in_lin, scale):
             elif in_lin(i, j):
                 w = 0.0
                 for a in range(d):
-                    fq = q[i, a] + 1 if q[i, a] > 0 else np.exp(q[i, a])
-                    fk = k[j, a] + 1 if k[j, a] > 0 else np.exp(k[j, a])
-                    w += fq * fk
+                    w += _phi_scalar(q[i, a], phi) * _phi_scalar(k[j, a], phi)
             else:
                 w = 0.0
             num += w * v[j]
@@ -86,18 +109,19 @@ def _bruteforce(q, k, v, in_soft, in_lin, scale):
     return out
 
 
-def test_bruteforce_bidir_window():
+@pytest.mark.parametrize("phi", ["elu1", "relu", "exp"])
+def test_bruteforce_bidir_window(phi):
     T, F, d = 5, 6, 4
     N = T * F
     q, k, v = (_rand((1, 1, N, d), s) for s in (7, 8, 9))
     C, h = 2, 1
-    o = oracle.bidir_window_attention(q, k, v, F, T, C, h)[0, 0]
+    o = oracle.bidir_window_attention(q, k, v, F, T, C, h, phi=phi)[0, 0]
 
     def soft(i, j):
         c = (i // F) // C
         return max(0, c * C - h) * F <= j < min(T, (c + 1) * C + h) * F
 
-    ref = _bruteforce(q[0, 0], k[0, 0], v[0, 0], soft, lambda i, j: not soft(i, j), 0.5)
+    ref = _bruteforce(q[0, 0], k[0, 0], v[0, 0], soft, lambda i, j: not soft(i, j), 0.5, phi)
     np.testing.assert_allclose(o, ref, rtol=1e-12)
 
 
