@@ -60,11 +60,19 @@ def peaks():
 
 
 # ----------------------------------------------------------------- work counts
+def workload_mask(w):
+    """The tile mask a block-mask workload runs with (None for the other modes)."""
+    from linear_attention_video_hyat_b200 import hyat
+    if w.mode == "lvsa":
+        return hyat.lvsa_mask(w.n_frames, w.tokens_per_frame, w.window_frames, w.anchor_stride, w.rotation)[None]
+    return None
+
+
 def work_counts(w):
     """Effective FLOPs of one call and the attention kernel's share, from the library layout."""
     from linear_attention_video_hyat_b200 import hyat
     cfg = hyat.config_from_workload(w)
-    work, ent = hyat.plan_layout(cfg)
+    work, ent = hyat.plan_layout(cfg, workload_mask(w))
     per_bh = work[work[:, 0] == 0]
     klen = np.concatenate([[0], np.cumsum(ent[:, 1].astype(np.int64))])
     pairs = int(sum(int(it[2]) * int(klen[it[5]] - klen[it[4]]) for it in per_bh))
@@ -174,6 +182,10 @@ def oracle_sample(w, n_blocks, rows_per_block=256, seed=0, qkv=None):
                                           w.halo_frames, rows=rows)
         elif w.mode == "radial":
             oracle.radial_attention(qs, ks, vs, w.n_frames, w.tokens_per_frame, rows=rows)
+        elif w.mode == "lvsa":
+            mask = oracle.lvsa_tile_mask(w.n_frames, w.tokens_per_frame, w.window_frames, w.anchor_stride,
+                                         w.rotation)[None]
+            oracle.blockmask_attention(qs, ks, vs, mask, rows=rows)
         else:
             raise ValueError("oracle timing covers the bidirectional workloads")
         t += time.perf_counter() - t0
@@ -368,11 +380,13 @@ def main():
     w = wl.WORKLOADS[a.workload]
     if w.mode == "stream":
         return bench_stream(a, w, rank, world, local)
-    assert w.mode in ("window", "radial"), "the bench times a bidirectional layer call or streaming steps"
+    assert w.mode in ("window", "radial", "lvsa"), "the bench times a bidirectional layer call or streaming steps"
     counts = work_counts(w)
     config = {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "tokens": w.N,
               "tokens_per_frame": w.tokens_per_frame, "frames": w.n_frames, "mode": w.mode,
               "chunk_frames": w.chunk_frames, "halo_frames": w.halo_frames,
+              **({"window_frames": w.window_frames, "anchor_stride": w.anchor_stride, "rotation": w.rotation}
+                 if w.mode == "lvsa" else {}),
               "parallelism": f"replicas{world}" if world > 1 else "single",
               "l2": "inputs larger than L2 (Q,K,V,O %.0f MB > 126 MB); no flush" % (4 * w.B * w.H * w.N * w.d * 2 / 1e6)}
 
@@ -410,7 +424,7 @@ def main():
     q, k, v = wl.gen_qkv(w, seed=w.seed + rank)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     od = torch.empty_like(qd)
-    h = hyat.Hyat(hyat.config_from_workload(w), device=dev)
+    h = hyat.Hyat(hyat.config_from_workload(w), workload_mask(w), device=dev)
     stream = torch.cuda.current_stream(dev)
     for _ in range(max(a.warmup, 3)):
         h.forward(qd, kd, vd, out=od)

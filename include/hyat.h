@@ -179,6 +179,20 @@ HYAT_API hyat_status hyat_plan_layout(const hyat_config* cfg, const uint8_t* hos
 HYAT_API hyat_status hyat_radial_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t* out,
                              size_t out_bytes);
 
+/* Host-only structured-window + rotating-anchor tile mask, for BLOCKMASK
+ * handles (Long Video Sparse Attention, Abstract: a structured window pattern
+ * with rotating global anchors). The pages do not define the pattern; this
+ * reading keeps tile (a, b) iff
+ *   - some query token of tile a and key token of tile b lie at most
+ *     (window_frames - 1) / 2 frames apart (window_frames odd), or
+ *   - tile b holds a token of an anchor frame f: (f + rotation) % anchor_stride
+ *     == 0 (anchor_stride 0: no anchors).
+ * The caller advances `rotation` (e.g. with the denoising step) so the anchor
+ * grid moves. Everything the mask drops reaches the query through the linear
+ * state. out = uint8 [nT, nT], nT = ceil(T*F/128). */
+HYAT_API hyat_status hyat_lvsa_mask(int32_t n_frames, int32_t tokens_per_frame, int32_t window_frames,
+                           int32_t anchor_stride, int32_t rotation, uint8_t* out, size_t out_bytes);
+
 /* Host-only streaming bookkeeping of step `step`: info[0] = first visible
  * chunk, info[1] = number of visible chunks, info[2] = chunk folded into the
  * state before this step's attention (-1 if none), info[3] = ring slot

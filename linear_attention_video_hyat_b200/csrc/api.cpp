@@ -536,6 +536,17 @@ hyat_status hyat_radial_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t
   return HYAT_OK;
 }
 
+hyat_status hyat_lvsa_mask(int32_t n_frames, int32_t tokens_per_frame, int32_t window_frames,
+                           int32_t anchor_stride, int32_t rotation, uint8_t* out, size_t out_bytes) {
+  if (n_frames < 1 || tokens_per_frame < 1 || !out || window_frames < 1 || window_frames % 2 == 0 ||
+      anchor_stride < 0 || rotation < 0)
+    return HYAT_ERR_INVALID_ARG;
+  const int64_t nT = tiles(int64_t(n_frames) * tokens_per_frame);
+  if (out_bytes < size_t(nT * nT)) return HYAT_ERR_INVALID_ARG;
+  lvsa_tile_mask(n_frames, tokens_per_frame, window_frames, anchor_stride, rotation, out);
+  return HYAT_OK;
+}
+
 hyat_status hyat_stream_plan(const hyat_config* cfg, int32_t step, int32_t* info, size_t info_len) {
   if (!cfg || !info || step < 0 || cfg->mode != HYAT_MODE_STREAM || !validate_config(*cfg).empty())
     return HYAT_ERR_INVALID_ARG;

@@ -67,6 +67,11 @@ bool prefer_split_pairs(size_t n_ordinary_pairs, int32_t num_sms);
 // build_pairs or build_split_pairs (by prefer_split_pairs), then order_pairs_for_grid.
 std::vector<int4> choose_pairs(const std::vector<WorkItem>& work, int32_t num_sms);
 void radial_tile_mask(int32_t n_frames, int32_t tokens_per_frame, uint8_t* out);
+// Structured window plus rotating global anchors on the 128-token tile grid: tile (a, b) is
+// kept iff some query token of a and key token of b are at most (window_frames - 1) / 2 frames
+// apart, or b holds a token of an anchor frame f ((f + rotation) % anchor_stride == 0).
+void lvsa_tile_mask(int32_t n_frames, int32_t tokens_per_frame, int32_t window_frames, int32_t anchor_stride,
+                    int32_t rotation, uint8_t* out);
 
 // ---- kernel launch wrappers (kernels_simt.cu, attn_tc.cu) ----
 struct SegStateArgs {

@@ -107,6 +107,29 @@ void radial_tile_mask(int32_t n_frames, int32_t F, uint8_t* out) {
   }
 }
 
+void lvsa_tile_mask(int32_t n_frames, int32_t F, int32_t window_frames, int32_t anchor_stride, int32_t rotation,
+                    uint8_t* out) {
+  const int64_t N = static_cast<int64_t>(n_frames) * F;
+  const int32_t nT = tiles(N);
+  const int32_t half = (window_frames - 1) / 2;
+  // frames covered by each tile, and whether a tile holds a token of an anchor frame
+  std::vector<int32_t> f_lo(nT), f_hi(nT);
+  std::vector<uint8_t> has_anchor(nT, 0);
+  for (int32_t t = 0; t < nT; ++t) {
+    const int64_t r0 = static_cast<int64_t>(t) * kTile, r1 = std::min<int64_t>(N, r0 + kTile) - 1;
+    f_lo[t] = static_cast<int32_t>(r0 / F);
+    f_hi[t] = static_cast<int32_t>(r1 / F);
+    if (anchor_stride > 0)
+      for (int32_t f = f_lo[t]; f <= f_hi[t]; ++f)
+        if ((f + rotation) % anchor_stride == 0) has_anchor[t] = 1;
+  }
+  for (int32_t a = 0; a < nT; ++a)
+    for (int32_t b = 0; b < nT; ++b) {
+      const int32_t gap = std::max(0, std::max(f_lo[b] - f_hi[a], f_lo[a] - f_hi[b]));
+      out[static_cast<size_t>(a) * nT + b] = (gap <= half || has_anchor[b]) ? 1 : 0;
+    }
+}
+
 static void push_window_entries(int64_t k_lo, int64_t k_hi, std::vector<Entry>* e) {
   for (int64_t k = k_lo; k < k_hi; k += kTile)
     e->push_back(Entry{static_cast<int32_t>(k), static_cast<int32_t>(std::min<int64_t>(kTile, k_hi - k))});

@@ -25,13 +25,15 @@ FLAG_TEST_DEVICE_TIMEOUT = 2
 TILE = 128
 KERNEL_KINDS = ("state", "complement", "attention", "fold_ring", "layout_prep")
 
-_MODES = {"window": MODE_WINDOW, "blockmask": MODE_BLOCKMASK, "radial": MODE_RADIAL, "stream": MODE_STREAM}
+_MODES = {"window": MODE_WINDOW, "blockmask": MODE_BLOCKMASK, "radial": MODE_RADIAL, "stream": MODE_STREAM,
+          "lvsa": MODE_BLOCKMASK}   # LVSA: a block mask from lvsa_mask()
 
 EXPORTED = (
     "hyat_workspace_bytes", "hyat_create", "hyat_fwd_bidir", "hyat_fwd_stream_step", "hyat_sync",
     "hyat_destroy", "hyat_last_error", "hyat_status_string", "hyat_plan_layout", "hyat_radial_mask",
     "hyat_stream_plan", "hyat_stream_state_bytes", "hyat_stream_get_state", "hyat_stream_set_state",
     "hyat_set_profiling", "hyat_kernel_times", "hyat_fwd_bidir_noalloc", "hyat_fwd_stream_denoise",
+    "hyat_lvsa_mask",
 )
 
 
@@ -71,6 +73,7 @@ def _load():
         "hyat_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "hyat_plan_layout": (ctypes.c_int, [CP, P, P, S, P, S, ctypes.POINTER(I64)]),
         "hyat_radial_mask": (ctypes.c_int, [I32, I32, P, S]),
+        "hyat_lvsa_mask": (ctypes.c_int, [I32, I32, I32, I32, I32, P, S]),
         "hyat_stream_plan": (ctypes.c_int, [CP, I32, P, S]),
         "hyat_stream_state_bytes": (S, [P]),
         "hyat_stream_get_state": (ctypes.c_int, [P, P, S]),
@@ -133,6 +136,16 @@ def plan_layout(cfg: Config, mask=None):
     _check(lib.hyat_plan_layout(ctypes.byref(cfg), mp, work.ctypes.data, work.size,
                                 ent.ctypes.data, ent.size, counts))
     return work, ent[:counts[1]]
+
+
+def lvsa_mask(n_frames: int, tokens_per_frame: int, window_frames: int, anchor_stride: int,
+              rotation: int = 0) -> np.ndarray:
+    """Structured-window + rotating-anchor tile mask (see hyat_lvsa_mask) for BLOCKMASK handles."""
+    nT = -(-n_frames * tokens_per_frame // TILE)
+    out = np.zeros((nT, nT), np.uint8)
+    _check(lib.hyat_lvsa_mask(n_frames, tokens_per_frame, window_frames, anchor_stride, rotation,
+                              out.ctypes.data, out.size))
+    return out
 
 
 def radial_mask(n_frames: int, tokens_per_frame: int) -> np.ndarray:

@@ -52,6 +52,8 @@ class Workload:
     per_head_std: bool = False
     seed: int = 0
     phi: str = "elu1"          # feature map of the linear branch: "elu1" | "relu" | "exp"
+    anchor_stride: int = 0     # lvsa only: every anchor_stride-th frame is a global anchor
+    rotation: int = 0          # lvsa only: shift of the anchor grid
     note: str = ""
 
     @property
@@ -93,7 +95,13 @@ RADIAL_84F = Workload(
     tokens_per_frame=1560, n_frames=84,
     note="84 latent frames x 1560 tokens, static radial tile mask")
 
-WORKLOADS = {w.name: w for w in (TINY_F32, WAN13B_BIDIR, WAN14B_BIDIR, STREAM_HF, RADIAL_84F)}
+LVSA_126F = Workload(
+    name="lvsa_T126x1560_w11_s4", mode="lvsa", B=1, H=12, d=128,
+    tokens_per_frame=1560, n_frames=126, window_frames=11, anchor_stride=4,
+    note="Wan-1.3B shapes at a 6x horizon (126 latent frames); structured window of 11 frames "
+         "plus every 4th frame as a global anchor (about a third of the tiles kept)")
+
+WORKLOADS = {w.name: w for w in (TINY_F32, WAN13B_BIDIR, WAN14B_BIDIR, STREAM_HF, RADIAL_84F, LVSA_126F)}
 
 
 def _cast(x: np.ndarray, w: Workload) -> torch.Tensor:

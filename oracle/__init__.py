@@ -20,6 +20,8 @@ from .hybrid import (  # noqa: F401
     radial_window,
     radial_token_near,
     radial_tile_mask,
+    lvsa_token_near,
+    lvsa_tile_mask,
     tile_mask_sets,
     stream_sets,
     stream_evicted_state,

@@ -259,6 +259,39 @@ def radial_tile_mask(n_frames, tokens_per_frame, tile=128):
     return mask
 
 
+# --------------------------------------------------------------------------
+# structured window + rotating global anchors (Long Video Sparse Attention,
+# Abstract). Reading (the pages give no rule): keys within (window_frames - 1)/2
+# frames of the query, plus every key of an anchor frame f with
+# (f + rotation) % anchor_stride == 0; a 128-token tile pair is kept iff it holds
+# such a token pair.
+# --------------------------------------------------------------------------
+def lvsa_token_near(i, j, tokens_per_frame, window_frames, anchor_stride, rotation):
+    """Token-level predicate (vectorised over broadcastable i, j)."""
+    fi = np.asarray(i, dtype=np.int64) // tokens_per_frame
+    fj = np.asarray(j, dtype=np.int64) // tokens_per_frame
+    near = np.abs(fi - fj) <= (window_frames - 1) // 2
+    if anchor_stride > 0:
+        near = near | ((fj + rotation) % anchor_stride == 0)
+    return near
+
+
+def lvsa_tile_mask(n_frames, tokens_per_frame, window_frames, anchor_stride, rotation=0, tile=128):
+    """Kept tiles [nT, nT] (uint8). A tile pair holds a near token pair iff the frames of
+    the two tiles come within the window, or the key tile touches an anchor frame."""
+    N = n_frames * tokens_per_frame
+    nT = -(-N // tile)
+    frames_of = [set(range((a * tile) // tokens_per_frame, (min(N, (a + 1) * tile) - 1) // tokens_per_frame + 1))
+                 for a in range(nT)]
+    half = (window_frames - 1) // 2
+    anchor = np.array([anchor_stride > 0 and any((f + rotation) % anchor_stride == 0 for f in fr)
+                       for fr in frames_of])
+    lo = np.array([min(fr) for fr in frames_of])
+    hi = np.array([max(fr) for fr in frames_of])
+    gap = np.maximum(0, np.maximum(lo[None, :] - hi[:, None], lo[:, None] - hi[None, :]))
+    return ((gap <= half) | anchor[None, :]).astype(np.uint8)
+
+
 def radial_attention(q, k, v, n_frames, tokens_per_frame, scale=None, rows=None,
                      tile=128, with_branches=False, phi="elu1"):
     mask = radial_tile_mask(n_frames, tokens_per_frame, tile)[None]

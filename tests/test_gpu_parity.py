@@ -351,8 +351,19 @@ def test_device_timeout_is_reported_and_recoverable():
 
 
 # ------------------------------------------------------------------ full-size workloads
+def _lvsa_masks(w):
+    """(library mask for the handle, oracle mask for the reference); equal bit for bit."""
+    lib_mask = hyat.lvsa_mask(w.n_frames, w.tokens_per_frame, w.window_frames, w.anchor_stride, w.rotation)
+    ref_mask = oracle.lvsa_tile_mask(w.n_frames, w.tokens_per_frame, w.window_frames, w.anchor_stride, w.rotation)
+    assert np.array_equal(lib_mask, ref_mask)
+    return lib_mask[None], ref_mask[None]
+
+
 def _bidir_sampled(w, heads, per_tile=2, seed=0):
-    o, (q, k, v) = _bidir(w)
+    lib_mask = ref_mask = None
+    if w.mode == "lvsa":
+        lib_mask, ref_mask = _lvsa_masks(w)
+    o, (q, k, v) = _bidir(w, mask=lib_mask)
     N = w.N
     if w.mode == "window":
         C = w.chunk_tokens
@@ -363,6 +374,8 @@ def _bidir_sampled(w, heads, per_tile=2, seed=0):
     qs, ks, vs = q[:, heads], k[:, heads], v[:, heads]
     if w.mode == "window":
         ref = _window_ref(w, qs, ks, vs, rows=rows)
+    elif w.mode == "lvsa":
+        ref = oracle.blockmask_attention(f64(qs), f64(ks), f64(vs), ref_mask, rows=rows)
     else:
         ref = oracle.radial_attention(f64(qs), f64(ks), f64(vs), w.n_frames, w.tokens_per_frame, rows=rows)
     got = f64(o[:, heads][:, :, rows])
@@ -385,6 +398,22 @@ def test_full_wan14b_bidir_sampled():
 def test_full_radial_sampled():
     got, ref = _bidir_sampled(wl.RADIAL_84F, heads=[0, 11], per_tile=2)
     assert_parity("bf16", got, ref, "radial")
+
+
+@pytest.mark.slow
+def test_full_lvsa_sampled():
+    got, ref = _bidir_sampled(wl.LVSA_126F, heads=[0, 7], per_tile=1)
+    assert_parity("bf16", got, ref, "lvsa")
+
+
+@pytest.mark.parametrize("wf,stride,rot", [(3, 3, 1), (5, 4, 0), (1, 2, 3)])
+def test_lvsa_small(wf, stride, rot):
+    w = wl.Workload("lvsa_small", "lvsa", 1, 2, 128, 300, 9, window_frames=wf, anchor_stride=stride,
+                    rotation=rot, seed=37)
+    lib_mask, ref_mask = _lvsa_masks(w)
+    o, (q, k, v) = _bidir(w, mask=lib_mask)
+    ref = oracle.blockmask_attention(f64(q), f64(k), f64(v), ref_mask)
+    assert_parity("bf16", f64(o), ref, (wf, stride, rot))
 
 
 @pytest.mark.slow

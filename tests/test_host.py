@@ -156,3 +156,20 @@ def test_peaked_bf16_bound_accepts_rounding_and_rejects_a_planted_error():
 def test_feature_maps_accepted(phi):
     cfg = hyat.make_config("window", 1, 2, 64, 64, 4, 1, 0, phi=phi)
     assert hyat.workspace_bytes(cfg) > 0
+
+
+@pytest.mark.parametrize("T,F,wf,stride,rot", [(21, 1560, 5, 4, 0), (21, 1560, 11, 3, 2), (126, 1560, 11, 4, 1),
+                                               (9, 300, 1, 0, 0), (7, 130, 3, 2, 5)])
+def test_lvsa_mask_matches_oracle(T, F, wf, stride, rot):
+    got = hyat.lvsa_mask(T, F, wf, stride, rot)
+    ref = oracle.lvsa_tile_mask(T, F, wf, stride, rot)
+    np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("bad", [dict(window_frames=4), dict(window_frames=0), dict(anchor_stride=-1),
+                                 dict(rotation=-1)])
+def test_lvsa_mask_rejects_bad_arguments(bad):
+    kw = dict(n_frames=5, tokens_per_frame=100, window_frames=3, anchor_stride=2, rotation=0)
+    kw.update(bad)
+    with pytest.raises(hyat.HyatError):
+        hyat.lvsa_mask(**kw)

@@ -351,3 +351,36 @@ def test_effective_pairs():
     assert oracle.effective_pairs_bidir(64, 4, 1, 0) == 4 * 64 ** 2
     tm = np.ones((1, 3, 3), np.uint8)
     assert oracle.effective_pairs_tile_mask(tm, 300, 300)[0] == 300 * 300
+
+
+# -------------------------------------------------------------- LVSA mask
+@pytest.mark.parametrize("F,T,wf,stride,rot", [(10, 7, 3, 3, 0), (10, 7, 1, 2, 1), (13, 5, 5, 0, 0), (6, 9, 3, 4, 2)])
+def test_lvsa_tile_mask_is_token_bruteforce(F, T, wf, stride, rot):
+    tile = 8
+    N = T * F
+    nT = -(-N // tile)
+    m = oracle.lvsa_tile_mask(T, F, wf, stride, rot, tile=tile)
+    for a in range(nT):
+        for b in range(nT):
+            i = np.arange(a * tile, min(N, (a + 1) * tile))[:, None]
+            j = np.arange(b * tile, min(N, (b + 1) * tile))[None, :]
+            # the predicate, evaluated from its definition with plain integer arithmetic
+            near = any((abs(ii // F - jj // F) <= (wf - 1) // 2) or (stride > 0 and (jj // F + rot) % stride == 0)
+                       for ii in i[:, 0] for jj in j[0])
+            assert m[a, b] == int(near), (a, b)
+    np.testing.assert_array_equal(
+        m, np.array([[int(oracle.lvsa_token_near(np.arange(a * tile, min(N, (a + 1) * tile))[:, None],
+                                                  np.arange(b * tile, min(N, (b + 1) * tile))[None, :],
+                                                  F, wf, stride, rot).any())
+                      for b in range(nT)] for a in range(nT)]))
+
+
+def test_lvsa_tile_mask_invariants():
+    T, F = 12, 50
+    base = oracle.lvsa_tile_mask(T, F, 3, 4, 1, tile=16)
+    np.testing.assert_array_equal(base, oracle.lvsa_tile_mask(T, F, 3, 4, 5, tile=16))   # period = stride
+    assert np.all(np.diag(base) == 1)                                                     # own tile always kept
+    assert np.all(oracle.lvsa_tile_mask(T, F, 2 * T + 1, 4, 1, tile=16) == 1)              # window covers all
+    win = oracle.lvsa_tile_mask(T, F, 3, 0, 0, tile=16)                                    # no anchors: banded
+    assert np.all(win == win.T)
+    assert base.sum() > win.sum()
