@@ -109,6 +109,8 @@ typedef struct {
   int32_t mask_heads;            /* BLOCKMASK / STREAM masks: 1 (shared) or H */
   uint32_t flags;                /* HYAT_FLAG_* */
   float scale;                   /* softmax logit scale; 0 => 1/sqrt(d) */
+  int32_t sink_frames;           /* STREAM: leading frames kept in the window for good (an
+                                    attention sink); a multiple of chunk_frames, 0 = none */
 } hyat_config;
 
 typedef struct hyat_ctx* hyat_handle;

@@ -54,12 +54,12 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
   p.entries = take(sizeof(Entry) * std::max<int64_t>(n_entries, 1));
   p.pairs = take(sizeof(int4) * std::max<int64_t>(n_work, 1));
   if (c.mode == HYAT_MODE_STREAM) {
-    const int64_t Lc = stream_chunk_tokens(c), nwc = stream_window_chunks(c), nqt = tiles(Lc);
+    const int64_t Lc = stream_chunk_tokens(c), slots = stream_ring_slots(c), nqt = tiles(Lc);
     p.srest = take(sizeof(float) * BH * E);
     p.srest_bf16 = take(2 * BH * c.d * c.d);
-    p.ring_k = take(size_t(BH * nwc * Lc * c.d * elem_bytes(c)));
-    p.ring_v = take(size_t(BH * nwc * Lc * c.d * elem_bytes(c)));
-    p.mask = take(size_t(c.mask_heads) * nqt * nqt * nwc);
+    p.ring_k = take(size_t(BH * slots * Lc * c.d * elem_bytes(c)));
+    p.ring_v = take(size_t(BH * slots * Lc * c.d * elem_bytes(c)));
+    p.mask = take(size_t(c.mask_heads) * nqt * nqt * slots);
     p.fold_partial = take(sizeof(float) * BH * fold_parts_cap(c) * E);
   } else {
     p.cm = take(sizeof(float) * size_t(L.cm_heads) * L.nqg * L.nseg);
@@ -80,7 +80,7 @@ bool plan_counts(const hyat_config& c, const uint8_t* host_mask, Layout* L, int6
     *err = build_layout(c, nullptr, L);
     const int64_t nqt = tiles(stream_chunk_tokens(c));
     *n_work = int64_t(c.B) * c.H * nqt;
-    *n_entries = *n_work * nqt * stream_window_chunks(c);
+    *n_entries = *n_work * nqt * stream_ring_slots(c);
     return err->empty();
   }
   if (c.mode == HYAT_MODE_BLOCKMASK && host_mask == nullptr) {
@@ -423,8 +423,8 @@ hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void*
   const hyat_config& c = h->cfg;
   const int32_t Lc = stream_chunk_tokens(c), nwc = stream_window_chunks(c), nqt = tiles(Lc);
   const int32_t s_ = h->step;
-  const int32_t first_visible = std::max(0, s_ - nwc + 1);
-  const int32_t nwin = s_ - first_visible + 1;
+  const StreamGeometry g = stream_geometry(c, s_);
+  const int32_t nwin = g.n_visible;
   const int32_t nkt = nqt * nwin;
   const size_t mask_bytes = size_t(c.mask_heads) * nqt * nkt;
   if (host_step_mask) {
@@ -441,10 +441,10 @@ hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void*
   else
     e = cudaMemsetAsync(h->d_mask, 1, mask_bytes, s);
   if (e != cudaSuccess) return cuda_fail(h, e, "step mask upload");
-  const int32_t slot = s_ % nwc;
-  const bool fold = s_ >= nwc && h->folded_step != s_;
+  const int32_t slot = g.write_slot;
+  const bool fold = g.evicted >= 0 && h->folded_step != s_;
   e = timed(h, K_FOLD, s, [&]() -> cudaError_t {
-    if (fold) {  // chunk s - nwc leaves the window: fold it into S, z
+    if (fold) {  // chunk s - nwc leaves the window: fold it into S, z (its slot is the one now written)
       SegStateArgs sa{};
       sa.k = h->d_ring_k; sa.v = h->d_ring_v; sa.rows_per_bh = h->rk;
       sa.BH = h->BH; sa.d = c.d; sa.dtype = c.dtype; sa.phi = c.phi;
@@ -467,7 +467,7 @@ hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void*
     }
     RingCopyArgs ra{};
     ra.k = k; ra.v = v; ra.ring_k = h->d_ring_k; ra.ring_v = h->d_ring_v;
-    ra.BH = h->BH; ra.L = Lc; ra.d = c.d; ra.nslots = nwc; ra.slot = slot;
+    ra.BH = h->BH; ra.L = Lc; ra.d = c.d; ra.nslots = stream_ring_slots(c); ra.slot = slot;
     ra.elem_bytes = static_cast<int32_t>(elem_bytes(c));
     return launch_ring_copy(ra, s);
   });
@@ -476,7 +476,8 @@ hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void*
   StreamLayoutArgs la{};
   la.mask = h->d_mask; la.work = h->d_work; la.entries = h->d_entries;
   la.BH = h->BH; la.H = c.H; la.mask_heads = c.mask_heads; la.nqt = nqt; la.nkt = nkt;
-  la.cap = nqt * nwc; la.L = Lc; la.nwc = nwc; la.first_visible = first_visible;
+  la.cap = nqt * stream_ring_slots(c); la.L = Lc; la.nwc = nwc;
+  la.n_sink_visible = g.n_sink_visible; la.first_window = g.first_window;
   e = timed(h, K_PREP, s, [&] { return launch_stream_layout(la, s); });
   if (e != cudaSuccess) return cuda_fail(h, e, "stream layout kernel");
   st = launch_attention(h, attn_args(h, q, h->d_ring_k, h->d_ring_v, o, int64_t(h->BH) * nqt, 1), s);
@@ -550,14 +551,17 @@ hyat_status hyat_lvsa_mask(int32_t n_frames, int32_t tokens_per_frame, int32_t w
 hyat_status hyat_stream_plan(const hyat_config* cfg, int32_t step, int32_t* info, size_t info_len) {
   if (!cfg || !info || step < 0 || cfg->mode != HYAT_MODE_STREAM || !validate_config(*cfg).empty())
     return HYAT_ERR_INVALID_ARG;
-  const int32_t nwc = stream_window_chunks(*cfg);
-  if (info_len < size_t(4 + nwc)) return HYAT_ERR_INVALID_ARG;
-  const int32_t first = std::max(0, step - nwc + 1);
-  info[0] = first;
-  info[1] = step - first + 1;
-  info[2] = step >= nwc ? step - nwc : -1;
-  info[3] = step % nwc;
-  for (int32_t w = 0; w < nwc; ++w) info[4 + w] = w < info[1] ? (first + w) % nwc : -1;
+  const int32_t slots = stream_ring_slots(*cfg);
+  if (info_len < size_t(4 + slots)) return HYAT_ERR_INVALID_ARG;
+  const StreamGeometry g = stream_geometry(*cfg, step);
+  info[0] = g.first_window;
+  info[1] = g.n_visible;
+  info[2] = g.evicted;
+  info[3] = g.write_slot;
+  for (int32_t w = 0; w < slots; ++w) {
+    const int32_t chunk = w < g.n_sink_visible ? w : g.first_window + (w - g.n_sink_visible);
+    info[4 + w] = w < g.n_visible ? stream_slot_of_chunk(*cfg, chunk) : -1;
+  }
   return HYAT_OK;
 }
 
@@ -566,14 +570,15 @@ namespace {
 struct StateHeader {
   uint32_t magic, version;
   int32_t step, BH, d, L, nwc, dtype;
-  int32_t folded_step, reserved[3];   // version 2: the step whose evicted chunk is in S, z
+  int32_t folded_step, reserved[3];   // version 2: the step whose evicted chunk is in S, z;
+                                      // reserved[0]: sink chunks
 };
 constexpr uint32_t kMagic = 0x54415948u;  // "HYAT"
 }  // namespace
 
 size_t hyat_stream_state_bytes(hyat_handle h) {
   if (!h || h->cfg.mode != HYAT_MODE_STREAM) return 0;
-  const size_t ring = size_t(h->BH) * stream_window_chunks(h->cfg) * stream_chunk_tokens(h->cfg) * h->cfg.d *
+  const size_t ring = size_t(h->BH) * stream_ring_slots(h->cfg) * stream_chunk_tokens(h->cfg) * h->cfg.d *
                       elem_bytes(h->cfg);
   return sizeof(StateHeader) + sizeof(float) * size_t(h->BH) * h->E + 2 * ring;
 }
@@ -585,7 +590,7 @@ hyat_status hyat_stream_get_state(hyat_handle h, void* dst_host, size_t bytes) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(h, e, "synchronize");
   StateHeader hd{kMagic, 2, h->step, h->BH, h->cfg.d, stream_chunk_tokens(h->cfg), stream_window_chunks(h->cfg),
-                 h->cfg.dtype, h->folded_step, {0, 0, 0}};
+                 h->cfg.dtype, h->folded_step, {stream_sink_chunks(h->cfg), 0, 0}};
   char* p = static_cast<char*>(dst_host);
   std::memcpy(p, &hd, sizeof(hd));
   p += sizeof(hd);
@@ -606,6 +611,7 @@ hyat_status hyat_stream_set_state(hyat_handle h, const void* src_host, size_t by
   std::memcpy(&hd, src_host, sizeof(hd));
   if (hd.magic != kMagic || hd.version != 2 || hd.BH != h->BH || hd.d != h->cfg.d ||
       hd.L != stream_chunk_tokens(h->cfg) || hd.nwc != stream_window_chunks(h->cfg) || hd.dtype != h->cfg.dtype ||
+      hd.reserved[0] != stream_sink_chunks(h->cfg) ||
       hd.step < 0 || hd.folded_step > hd.step)
     return fail(h, HYAT_ERR_STATE, "state blob does not match this handle");
   cudaError_t e = cudaDeviceSynchronize();

@@ -46,7 +46,18 @@ std::string validate_config(const hyat_config& c);
 int64_t rows_q(const hyat_config& c);           // query rows per (b, h)
 int64_t rows_k(const hyat_config& c);           // key rows per (b, h) (ring for STREAM)
 int32_t stream_chunk_tokens(const hyat_config& c);
-int32_t stream_window_chunks(const hyat_config& c);
+int32_t stream_window_chunks(const hyat_config& c);   // rolling window, in chunks
+int32_t stream_sink_chunks(const hyat_config& c);     // leading chunks kept for good
+int32_t stream_ring_slots(const hyat_config& c);      // window + sink slots per (b, h)
+// Chunks visible at a streaming step: the sink chunks [0, n_sink_visible) first, then the
+// rolling window [first_window, step]; key tiles follow that order.
+struct StreamGeometry {
+  int32_t n_sink_visible, first_window, n_window, n_visible;
+  int32_t evicted;      // chunk folded into S, z at this step (-1: none)
+  int32_t write_slot;   // ring slot of this step's chunk
+};
+StreamGeometry stream_geometry(const hyat_config& c, int32_t step);
+int32_t stream_slot_of_chunk(const hyat_config& c, int32_t chunk);
 int32_t tiles(int64_t rows);
 
 // Host layout builders (layout.cpp).
@@ -163,7 +174,9 @@ struct StreamLayoutArgs {
   const uint8_t* mask;            // [mask_heads][nqt][nkt] (device)
   WorkItem* work;                 // [BH][nqt]
   Entry* entries;                 // [BH][nqt][cap]
-  int32_t BH, H, mask_heads, nqt, nkt, cap, L, nwc, first_visible;
+  int32_t BH, H, mask_heads, nqt, nkt, cap, L, nwc;
+  int32_t n_sink_visible;         // visible chunks 0..n_sink_visible-1 sit in slots nwc + c
+  int32_t first_window;           // the following visible chunks c >= first_window: slot c % nwc
 };
 cudaError_t launch_stream_layout(const StreamLayoutArgs& a, cudaStream_t s);
 

@@ -226,7 +226,7 @@ __global__ void stream_layout_kernel(StreamLayoutArgs a) {
     if (keep) {
       const int pos = count + __popc(bal & ((1u << lane) - 1u));
       const int w = kt / a.nqt, t = kt % a.nqt;
-      const int slot = (a.first_visible + w) % a.nwc;
+      const int slot = w < a.n_sink_visible ? a.nwc + w : (a.first_window + w - a.n_sink_visible) % a.nwc;
       a.entries[base + pos] = Entry{slot * a.L + t * kTile, min(kTile, a.L - t * kTile)};
     }
     count += __popc(bal);

@@ -18,6 +18,25 @@ int32_t tiles(int64_t rows) { return static_cast<int32_t>((rows + kTile - 1) / k
 
 int32_t stream_chunk_tokens(const hyat_config& c) { return c.chunk_frames * c.tokens_per_frame; }
 int32_t stream_window_chunks(const hyat_config& c) { return c.window_frames / c.chunk_frames; }
+int32_t stream_sink_chunks(const hyat_config& c) { return c.sink_frames / c.chunk_frames; }
+int32_t stream_ring_slots(const hyat_config& c) { return stream_window_chunks(c) + stream_sink_chunks(c); }
+
+StreamGeometry stream_geometry(const hyat_config& c, int32_t step) {
+  StreamGeometry g;
+  const int32_t nwc = stream_window_chunks(c), ns = stream_sink_chunks(c);
+  g.n_sink_visible = std::min(ns, step + 1);
+  g.first_window = std::max(ns, step - nwc + 1);
+  g.n_window = step >= g.first_window ? step - g.first_window + 1 : 0;
+  g.n_visible = g.n_sink_visible + g.n_window;
+  g.evicted = step - nwc >= ns ? step - nwc : -1;
+  g.write_slot = stream_slot_of_chunk(c, step);
+  return g;
+}
+
+int32_t stream_slot_of_chunk(const hyat_config& c, int32_t chunk) {
+  const int32_t nwc = stream_window_chunks(c);
+  return chunk < stream_sink_chunks(c) ? nwc + chunk : chunk % nwc;
+}
 
 int64_t rows_q(const hyat_config& c) {
   if (c.mode == HYAT_MODE_STREAM) return stream_chunk_tokens(c);
@@ -26,7 +45,7 @@ int64_t rows_q(const hyat_config& c) {
 
 int64_t rows_k(const hyat_config& c) {
   if (c.mode == HYAT_MODE_STREAM)
-    return static_cast<int64_t>(stream_window_chunks(c)) * stream_chunk_tokens(c);
+    return static_cast<int64_t>(stream_ring_slots(c)) * stream_chunk_tokens(c);
   return static_cast<int64_t>(c.n_frames) * c.tokens_per_frame;
 }
 
@@ -56,6 +75,8 @@ std::string validate_config(const hyat_config& c) {
       if (c.window_frames < c.chunk_frames || c.window_frames % c.chunk_frames != 0)
         return "window_frames must be a positive multiple of chunk_frames";
       if (c.mask_heads != 1 && c.mask_heads != c.H) return "mask_heads must be 1 or H";
+      if (c.sink_frames < 0 || c.sink_frames % c.chunk_frames != 0)
+        return "sink_frames must be a non-negative multiple of chunk_frames";
       break;
     default:
       return "unknown mode";

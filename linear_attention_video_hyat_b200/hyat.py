@@ -50,7 +50,7 @@ class Config(ctypes.Structure):
         ("chunk_frames", ctypes.c_int32), ("halo_frames", ctypes.c_int32),
         ("window_frames", ctypes.c_int32), ("mode", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("phi", ctypes.c_int32), ("mask_heads", ctypes.c_int32), ("flags", ctypes.c_uint32),
-        ("scale", ctypes.c_float),
+        ("scale", ctypes.c_float), ("sink_frames", ctypes.c_int32),
     ]
 
 
@@ -96,18 +96,19 @@ PHI = {"elu1": 0, "relu": 1, "exp": 2}   # hyat_phi
 
 
 def make_config(mode, B, H, d, tokens_per_frame, n_frames=0, chunk_frames=1, halo_frames=0,
-                window_frames=0, dtype=BF16, mask_heads=1, flags=0, scale=0.0, phi="elu1") -> Config:
+                window_frames=0, dtype=BF16, mask_heads=1, flags=0, scale=0.0, phi="elu1",
+                sink_frames=0) -> Config:
     m = _MODES[mode] if isinstance(mode, str) else int(mode)
     dt = {"f32": F32, "bf16": BF16}.get(dtype, dtype) if isinstance(dtype, str) else int(dtype)
     ph = PHI[phi] if isinstance(phi, str) else int(phi)
     return Config(B, H, d, tokens_per_frame, n_frames, chunk_frames, halo_frames, window_frames,
-                  m, dt, ph, mask_heads, flags, float(scale))
+                  m, dt, ph, mask_heads, flags, float(scale), int(sink_frames))
 
 
 def config_from_workload(w, flags=0, mask_heads=1) -> Config:
     return make_config(w.mode, w.B, w.H, w.d, w.tokens_per_frame, w.n_frames, w.chunk_frames,
                        w.halo_frames, w.window_frames, w.dtype, mask_heads=mask_heads, flags=flags,
-                       phi=getattr(w, "phi", "elu1"))
+                       phi=getattr(w, "phi", "elu1"), sink_frames=getattr(w, "sink_frames", 0))
 
 
 def _check(status, handle=None):
@@ -156,7 +157,7 @@ def radial_mask(n_frames: int, tokens_per_frame: int) -> np.ndarray:
 
 
 def stream_plan(cfg: Config, step: int):
-    nwc = cfg.window_frames // cfg.chunk_frames
+    nwc = cfg.window_frames // cfg.chunk_frames + cfg.sink_frames // cfg.chunk_frames   # ring slots
     info = np.zeros(4 + nwc, np.int32)
     _check(lib.hyat_stream_plan(ctypes.byref(cfg), step, info.ctypes.data, info.size))
     return {"first_visible": int(info[0]), "n_visible": int(info[1]), "evicted": int(info[2]),

@@ -52,6 +52,7 @@ class Workload:
     per_head_std: bool = False
     seed: int = 0
     phi: str = "elu1"          # feature map of the linear branch: "elu1" | "relu" | "exp"
+    sink_frames: int = 0       # stream only: leading frames kept in the window for good
     anchor_stride: int = 0     # lvsa only: every anchor_stride-th frame is a global anchor
     rotation: int = 0          # lvsa only: shift of the anchor grid
     note: str = ""
@@ -129,8 +130,13 @@ def stream_tiles_per_chunk(w: Workload) -> int:
 
 
 def stream_window_chunks(w: Workload, step: int) -> int:
-    """Number of chunks visible at ``step`` (the window holds window_frames frames)."""
-    return min(step + 1, w.window_frames // w.chunk_frames)
+    """Number of chunks visible at ``step``: the sink chunks (sink_frames) that exist, then
+    the rolling window of window_frames frames."""
+    n_sink = w.sink_frames // w.chunk_frames
+    nwc = w.window_frames // w.chunk_frames
+    if step < n_sink:
+        return step + 1
+    return n_sink + min(step - n_sink + 1, nwc)
 
 
 def gen_stream_step(w: Workload, step: int, seed: Optional[int] = None, keep_prob: float = 0.5,

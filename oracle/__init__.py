@@ -24,6 +24,7 @@ from .hybrid import (  # noqa: F401
     lvsa_tile_mask,
     tile_mask_sets,
     stream_sets,
+    stream_visible_chunks,
     stream_evicted_state,
     bidir_window_attention,
     blockmask_attention,

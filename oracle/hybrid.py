@@ -302,7 +302,15 @@ def radial_attention(q, k, v, n_frames, tokens_per_frame, scale=None, rows=None,
 # streaming (Hybrid Forcing §2.A: evicted frames feed a linear state; the
 # recent window is block-sparse softmax)
 # --------------------------------------------------------------------------
-def stream_sets(h, rows, step, chunk_tokens, n_window_chunks, tile_mask, tile=128):
+def stream_visible_chunks(step, n_window_chunks, n_sink_chunks=0):
+    """Chunks visible at ``step``, oldest first: the sink chunks that exist, then the latest
+    n_window_chunks chunks after them."""
+    sinks = list(range(min(n_sink_chunks, step + 1)))
+    first = max(n_sink_chunks, step - n_window_chunks + 1)
+    return sinks + list(range(first, step + 1))
+
+
+def stream_sets(h, rows, step, chunk_tokens, n_window_chunks, tile_mask, tile=128, n_sink_chunks=0):
     """Sets for query rows (chunk-local) of chunk ``step`` over keys of chunks 0..step.
 
     Key j is the global token index over the generated chunks; the mask is
@@ -312,12 +320,13 @@ def stream_sets(h, rows, step, chunk_tokens, n_window_chunks, tile_mask, tile=12
     hm = 0 if tm.shape[0] == 1 else h
     rows = np.asarray(rows, dtype=np.int64)
     nqt = -(-chunk_tokens // tile)
-    first_visible = max(0, step - n_window_chunks + 1)
+    vis = stream_visible_chunks(step, n_window_chunks, n_sink_chunks)
+    rank = {c: r for r, c in enumerate(vis)}
     n_keys = (step + 1) * chunk_tokens
     j = np.arange(n_keys)
     c_of_j = j // chunk_tokens
-    kt_of_j = (c_of_j - first_visible) * nqt + (j % chunk_tokens) // tile
-    visible = c_of_j >= first_visible
+    visible = np.isin(c_of_j, vis)
+    kt_of_j = np.array([rank.get(int(c), 0) for c in c_of_j], dtype=np.int64) * nqt + (j % chunk_tokens) // tile
     soft = np.zeros((len(rows), n_keys), dtype=bool)
     soft[:, visible] = tm[hm][rows // tile][:, kt_of_j[visible]]
     lin = np.broadcast_to(~visible, soft.shape).copy()
@@ -325,22 +334,25 @@ def stream_sets(h, rows, step, chunk_tokens, n_window_chunks, tile_mask, tile=12
 
 
 def stream_step_attention(q_chunk, k_hist, v_hist, step, chunk_tokens, n_window_chunks,
-                          tile_mask, scale=None, rows=None, tile=128, with_branches=False, phi="elu1"):
+                          tile_mask, scale=None, rows=None, tile=128, with_branches=False, phi="elu1",
+                          n_sink_chunks=0):
     """Output of chunk ``step``; k_hist, v_hist hold chunks 0..step ([B,H,(step+1)L,d])."""
     assert k_hist.shape[2] == (step + 1) * chunk_tokens
     sc = _default_scale(q_chunk.shape[-1], scale)
-    fn = lambda h, rr: stream_sets(h, rr, step, chunk_tokens, n_window_chunks, tile_mask, tile)
+    fn = lambda h, rr: stream_sets(h, rr, step, chunk_tokens, n_window_chunks, tile_mask, tile, n_sink_chunks)
     return _run_rows(q_chunk, k_hist, v_hist, rows, fn, sc, with_branches, phi)
 
 
-def stream_evicted_state(k_hist, v_hist, step, chunk_tokens, n_window_chunks, phi="elu1"):
-    """Linear state used at ``step``: S = sum phi(k) v^T, z = sum phi(k) over evicted chunks.
+def stream_evicted_state(k_hist, v_hist, step, chunk_tokens, n_window_chunks, phi="elu1", n_sink_chunks=0):
+    """Linear state used at ``step``: S = sum phi(k) v^T, z = sum phi(k) over evicted chunks
+    (chunks that are neither sinks nor in the window).
 
     Returns S [B,H,d,d] and z [B,H,d] in float64 (zero before anything is evicted).
     """
-    n_evicted = max(0, step - n_window_chunks + 1) * chunk_tokens
-    k = np.asarray(k_hist[:, :, :n_evicted], dtype=np.float64)
-    v = np.asarray(v_hist[:, :, :n_evicted], dtype=np.float64)
+    lo = n_sink_chunks * chunk_tokens
+    hi = max(n_sink_chunks, step - n_window_chunks + 1) * chunk_tokens
+    k = np.asarray(k_hist[:, :, lo:hi], dtype=np.float64)
+    v = np.asarray(v_hist[:, :, lo:hi], dtype=np.float64)
     pk = feature_map(phi)(k)
     S = np.einsum("bhna,bhnc->bhac", pk, v)
     z = pk.sum(axis=2)

@@ -262,6 +262,43 @@ def test_stream_checkpoint_between_denoising_calls_bit_identical():
     h2.close()
 
 
+def test_stream_with_attention_sink():
+    """The first chunk stays in the window for good; the chunks between it and the rolling
+    window are folded into the state; denoising calls see the sink too."""
+    w = wl.Workload("stream_sink", "stream", 1, 2, 128, 200, 27, chunk_frames=3, window_frames=6,
+                    n_steps=8, seed=41, sink_frames=3)
+    h = hyat.Hyat(hyat.config_from_workload(w, mask_heads=2))
+    L, nwc, ns = w.chunk_tokens, 2, 1
+    kh, vh = [], []
+    for s in range(8):
+        if s in (2, 5):
+            q, k, v, mask = wl.gen_stream_step(w, s, call=0)
+            o = h.stream_denoise(*_dev(q, k, v), mask=mask)
+            h.sync()
+            ref = oracle.stream_step_attention(f64(q), np.concatenate(kh + [k.float().numpy()], axis=2),
+                                               np.concatenate(vh + [v.float().numpy()], axis=2), s, L, nwc,
+                                               mask, n_sink_chunks=ns)
+            assert_parity("bf16", f64(o), ref, f"denoising call, chunk {s}")
+        q, k, v, mask = wl.gen_stream_step(w, s)
+        assert mask.shape[2] == (-(-L // 128)) * len(oracle.stream_visible_chunks(s, nwc, ns))
+        o = h.stream_step(*_dev(q, k, v), mask=mask)
+        h.sync()
+        kh.append(k.float().numpy())
+        vh.append(v.float().numpy())
+        ref = oracle.stream_step_attention(f64(q), np.concatenate(kh, axis=2), np.concatenate(vh, axis=2),
+                                           s, L, nwc, mask, n_sink_chunks=ns)
+        assert_parity("bf16", f64(o), ref, f"chunk {s}")
+    step, S, z = _state_from_blob(h.get_state(), 2, 128)
+    assert step == 8
+    k_all, v_all = np.concatenate(kh, axis=2), np.concatenate(vh, axis=2)
+    S_ref, z_ref = oracle.stream_evicted_state(k_all, v_all, 7, L, nwc, n_sink_chunks=ns)   # chunks 1..5
+    pk = oracle.phi_elu1(k_all[:, :, L:6 * L])
+    bound_S = 2.0 ** -8 * np.einsum("bhna,bhnc->bhac", pk, np.abs(v_all[:, :, L:6 * L]))
+    assert np.all(np.abs(S.reshape(1, 2, 128, 128) - S_ref) <= bound_S + 1e-5 * np.abs(S_ref).max())
+    assert np.all(np.abs(z.reshape(1, 2, 128) - z_ref) <= 2.0 ** -8 * pk.sum(axis=2) + 1e-5 * np.abs(z_ref).max())
+    h.close()
+
+
 # ------------------------------------------------------------------ feature maps
 @pytest.mark.parametrize("phi", ["relu", "exp"])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])

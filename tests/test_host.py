@@ -173,3 +173,24 @@ def test_lvsa_mask_rejects_bad_arguments(bad):
     kw.update(bad)
     with pytest.raises(hyat.HyatError):
         hyat.lvsa_mask(**kw)
+
+
+@pytest.mark.parametrize("sink_frames", [3, 6])
+def test_stream_plan_with_sink(sink_frames):
+    """Sink chunks keep their own slots for good; the rolling window cycles the others."""
+    w = wl.STREAM_HF.with_(sink_frames=sink_frames)
+    cfg = hyat.config_from_workload(w)
+    nwc, ns = 3, sink_frames // 3
+    slot_of = {}
+    for s in range(20):
+        p = hyat.stream_plan(cfg, s)
+        vis = oracle.stream_visible_chunks(s, nwc, ns)
+        assert p["n_visible"] == len(vis) == wl.stream_window_chunks(w, s)
+        assert p["first_visible"] == max(ns, s - nwc + 1)
+        assert p["evicted"] == (s - nwc if s - nwc >= ns else -1)
+        if p["evicted"] >= 0:
+            assert slot_of[p["evicted"]] == p["write_slot"]
+        slot_of[s] = p["write_slot"]
+        assert p["slots"] == [slot_of[c] for c in vis]
+        assert len(set(p["slots"])) == len(vis)
+        assert all(slot_of[c] == nwc + c for c in range(min(ns, s + 1)))

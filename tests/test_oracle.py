@@ -160,6 +160,35 @@ def test_bruteforce_stream_step():
     np.testing.assert_allclose(o, ref, rtol=1e-12)
 
 
+def test_bruteforce_stream_step_with_sink():
+    """Sink chunk 0 stays visible; chunk 1 is evicted; chunks 2, 3 form the window."""
+    L, d, tile, nwin, n_sink = 10, 4, 4, 2, 1
+    nqt = -(-L // tile)
+    step = 3
+    rng = np.random.default_rng(17)
+    kh, vh = rng.standard_normal((1, 1, 4 * L, d)), rng.standard_normal((1, 1, 4 * L, d))
+    qc = rng.standard_normal((1, 1, L, d))
+    vis = [0, 2, 3]
+    assert oracle.stream_visible_chunks(step, nwin, n_sink) == vis
+    mask = (rng.random((1, nqt, nqt * len(vis))) < 0.5).astype(np.uint8)
+    mask[0, np.arange(nqt), nqt * 2 + np.arange(nqt)] = 1
+    o = oracle.stream_step_attention(qc, kh, vh, step, L, nwin, mask, tile=tile, n_sink_chunks=n_sink)[0, 0]
+
+    def soft(i, j):
+        c = j // L
+        if c not in vis:
+            return False
+        return bool(mask[0, i // tile, vis.index(c) * nqt + (j % L) // tile])
+
+    ref = _bruteforce(qc[0, 0], kh[0, 0], vh[0, 0], soft, lambda i, j: j // L == 1, 0.5)
+    np.testing.assert_allclose(o, ref, rtol=1e-12)
+    # the evicted state holds chunk 1 only
+    S, z = oracle.stream_evicted_state(kh, vh, step, L, nwin, n_sink_chunks=n_sink)
+    pk = np.where(kh[0, 0, L:2 * L] > 0, kh[0, 0, L:2 * L] + 1, np.exp(kh[0, 0, L:2 * L]))
+    np.testing.assert_allclose(S[0, 0], pk.T @ vh[0, 0, L:2 * L], rtol=1e-13)
+    np.testing.assert_allclose(z[0, 0], pk.sum(0), rtol=1e-13)
+
+
 # ------------------------------------------------------------- closed forms
 def _frame_indicator_v(T, F, d):
     v = np.zeros((1, 1, T * F, d))
