@@ -63,18 +63,19 @@ struct StateParams {
   int32_t phi;               // feature map (hyat_phi)
 };
 
+// Bounded wait. After one plain probe the thread lets the hardware suspend it until the phase
+// completes (at most 1 ms per try), so waiting warps do not poll shared memory while the
+// TMA engine fills it.
 __device__ __forceinline__ bool swait(uint64_t* b, uint32_t parity, StateSmem* sm, uint32_t* status) {
   if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*reinterpret_cast<volatile int32_t*>(&sm->abort_flag)) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
-        atomicOr(status, kStatusTimeout);
-        *reinterpret_cast<volatile int32_t*>(&sm->abort_flag) = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_suspend(b, parity, 1000000u)) return true;
+    if (*reinterpret_cast<volatile int32_t*>(&sm->abort_flag)) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      atomicOr(status, kStatusTimeout);
+      *reinterpret_cast<volatile int32_t*>(&sm->abort_flag) = 1;
+      return false;
     }
   }
 }
