@@ -11,7 +11,9 @@
 // layout, so no transpose is needed:
 //   * warp 8 streams 64-token K and V tiles through a 6-stage ring (about 160 KB in
 //     flight per SM, enough to cover loaded-HBM latency);
-//   * warps 0-3 apply phi in place in shared memory (zeroing rows past the segment end);
+//   * warps 0-3 and 10-13 apply phi in place in shared memory, 32 rows of a stage each
+//     (zeroing rows past the segment end); loads, arithmetic and stores are batched so
+//     the chunks of a thread overlap;
 //   * warp 9 issues tcgen05.mma into a double-buffered TMEM accumulator; z comes from a
 //     second MMA against an all-ones 16-column operand (N = 16), so it costs no CUDA-core work;
 //   * warps 4-7 drain the accumulator of a finished segment to HBM while the next segment
@@ -31,7 +33,8 @@ constexpr int NST = 6;
 constexpr int KT_BYTES = TOK * D * 2;            // one [64 tokens x 128 features] bf16 tile
 constexpr int KT_HALF = KT_BYTES / 2;            // 64 features (128-byte rows)
 constexpr int STAGE_BYTES = 2 * KT_BYTES;        // K tile, then V tile
-constexpr int ST_THREADS = 320;                  // warps 0-3 phi, 4-7 drain, 8 TMA, 9 MMA
+constexpr int ST_THREADS = 448;                  // warps 0-3, 10-13 phi; 4-7 drain; 8 TMA; 9 MMA
+constexpr int PHI_THREADS = 256;                 // two phi warpgroups, 32 rows of a stage each
 constexpr int ST_TMA_WARP = 8, ST_MMA_WARP = 9;
 
 // D f32, A and B bf16 MN-major, M = 128, N = 128
@@ -111,9 +114,11 @@ __device__ __forceinline__ Unit unit_of(const StateParams& p, int u) {
 // zero), then hand the stage to the MMA warp.
 template <int kKind>
 __device__ __forceinline__ void phi_role(StateSmem* sm, const StateParams& p) {
-  // phi in place: thread t owns column chunk t % 16 of rows t / 16 + 8 k
-  const int t = threadIdx.x;
+  // phi in place: thread t of warpgroup g owns column chunk t % 16 of rows 32 g + t / 16 + 8 k
+  const int g = threadIdx.x >= 128 ? 1 : 0;                  // warps 0-3: g = 0; warps 10-13: g = 1
+  const int t = threadIdx.x - (g ? 320 : 0);
   const int cc = t & 15, half = cc >> 3, c8 = cc & 7;
+  const int row0 = 32 * g + (t >> 4);
   int st = 0;
   uint32_t ph = 0;
   bool ok = true;
@@ -123,23 +128,30 @@ __device__ __forceinline__ void phi_role(StateSmem* sm, const StateParams& p) {
       if (!(ok = swait_warp(&sm->full[st], ph, sm, p.status))) break;
       const int valid = x.len - TOK * i;
       uint8_t* kt = sm->stage[st] + half * KT_HALF;
-#pragma unroll 4
-      for (int k = 0; k < TOK / 8; ++k) {
-        const int r = (t >> 4) + 8 * k;
-        uint4* addr = reinterpret_cast<uint4*>(kt + r * 128 + ((c8 ^ (r & 7)) << 4));
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
-        if (r < valid) {
-          const uint4 raw = *addr;
-          const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t o4[4];
+      // all loads first, then the arithmetic, then all stores: the chunks are independent, and
+      // without this order every store would wait for the next load's address check
+      uint4 raw[TOK / 16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
-            o4[e] = pack_bf16(phi_of<kKind>(f.x), phi_of<kKind>(f.y));
-          }
-          w = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+      for (int k = 0; k < TOK / 16; ++k) {
+        const int r = row0 + 8 * k;
+        raw[k] = *reinterpret_cast<const uint4*>(kt + r * 128 + ((c8 ^ (r & 7)) << 4));
+      }
+#pragma unroll
+      for (int k = 0; k < TOK / 16; ++k) {
+        const int r = row0 + 8 * k;
+        const uint32_t in[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[e]));
+          o4[e] = pack_bf16(phi_of<kKind>(f.x), phi_of<kKind>(f.y));
         }
-        *addr = w;
+        raw[k] = r < valid ? make_uint4(o4[0], o4[1], o4[2], o4[3]) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < TOK / 16; ++k) {
+        const int r = row0 + 8 * k;
+        *reinterpret_cast<uint4*>(kt + r * 128 + ((c8 ^ (r & 7)) << 4)) = raw[k];
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&sm->phi_done[st]);
@@ -235,7 +247,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(&sm->full[i], 1);
-      mbar_init(&sm->phi_done[i], 128);
+      mbar_init(&sm->phi_done[i], PHI_THREADS);
       mbar_init(&sm->empty[i], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -321,7 +333,7 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
       while (!mbar_try_wait(&sm->drain, 0) && globaltimer() - t0 < kTimeoutNs) {
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 4 || warp >= 10) {
     if (p.phi == 1) phi_role<1>(sm, p);
     else if (p.phi == 2) phi_role<2>(sm, p);
     else phi_role<0>(sm, p);
