@@ -45,18 +45,18 @@ struct GemmParams {
   uint32_t* status;
 };
 
+// Bounded wait; after one plain probe the hardware may suspend the thread until the phase
+// completes (at most 1 ms per try), so waiting warps do not poll shared memory.
 __device__ __forceinline__ bool gwait(uint64_t* b, uint32_t parity, GemmSmem* sm, uint32_t* status) {
   if (mbar_try_wait(b, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*reinterpret_cast<volatile int32_t*>(&sm->abort_flag)) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
-        atomicOr(status, kStatusTimeout);
-        *reinterpret_cast<volatile int32_t*>(&sm->abort_flag) = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_suspend(b, parity, 1000000u)) return true;
+    if (*reinterpret_cast<volatile int32_t*>(&sm->abort_flag)) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      atomicOr(status, kStatusTimeout);
+      *reinterpret_cast<volatile int32_t*>(&sm->abort_flag) = 1;
+      return false;
     }
   }
 }
@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    // the whole warp runs the MMA role (warp-uniform descriptors); one elected lane issues
+    {
       int st = 0, c = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -136,10 +137,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++c) {
         const int buf = c & 1;
         const uint32_t tacc = tmem + buf * 128;
-        if (!(ok = gwait(&sm->acc_empty[buf], ((c >> 1) & 1) ^ 1u, sm, p.status))) break;
+        if (!(ok = __all_sync(0xffffffffu, gwait(&sm->acc_empty[buf], ((c >> 1) & 1) ^ 1u, sm, p.status)))) break;
         tc_fence_after();
         for (int kt = 0; kt < p.n_kt && ok; ++kt) {
-          if (!(ok = gwait(&sm->full[st], ph, sm, p.status))) break;
+          if (!(ok = __all_sync(0xffffffffu, gwait(&sm->full[st], ph, sm, p.status)))) break;
           tc_fence_after();
           const uint64_t da = dA0 + static_cast<uint64_t>(st) * kStage;
           const uint64_t dhi = dB0 + static_cast<uint64_t>(st) * kStage, dlo = dhi + kPart;
@@ -147,18 +148,19 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t a = da + static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
             const uint64_t bo = static_cast<uint64_t>(kk * (2048 >> 4));
-            mma_ss(tacc, a, dhi + bo, kIdescGemm, (kt | kk) != 0);
-            mma_ss(tacc, a, dlo + bo, kIdescGemm, 1);
+            mma_ss_elect(tacc, a, dhi + bo, kIdescGemm, (kt | kk) != 0);
+            mma_ss_elect(tacc, a, dlo + bo, kIdescGemm, 1);
           }
-          mma_commit(&sm->empty[st]);
+          mma_commit_elect(&sm->empty[st]);
           if (++st == G_NST) { st = 0; ph ^= 1u; }
         }
-        if (ok) mma_commit(&sm->acc_full[buf]);
+        if (ok) mma_commit_elect(&sm->acc_full[buf]);
       }
-      mma_commit(&sm->drain);
+      mma_commit_elect(&sm->drain);
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(&sm->drain, 0) && globaltimer() - t0 < kTimeoutNs) {
       }
+      __syncwarp();
     }
   } else if (warp >= 4) {
     const int rowl = (warp & 3) * 32 + lane;          // TMEM lane = group within the tile
