@@ -12,7 +12,10 @@
 //
 // Design for B200:
 //   * one persistent CTA per SM; a CTA owns a pair of 128-row query tiles
-//     ("slots"), so the softmax of one slot overlaps the MMAs of the other;
+//     ("slots"), so the softmax of one slot overlaps the MMAs of the other.
+//     Pairs are dealt largest first in a serpentine over the grid; when that
+//     would leave few waves, a "split pair" runs one query tile on both slots,
+//     each over half of its key tiles, and slot 0 merges the halves;
 //   * warp 8 issues TMA loads (Q tiles, K/V tiles, bf16 S_rest) into 128B-swizzled
 //     shared memory through a 5-stage ring; warp 9 issues tcgen05.mma (the
 //     whole warp runs the role, one elected lane issues) with fp32 accumulators
@@ -25,7 +28,8 @@
 //     moves (with a rescale of O in TMEM) only when the running sum would leave
 //     the safe fp32 range, which keeps the result exact and the rescale rare;
 //   * every mbarrier wait is bounded (%globaltimer); a wait that gives up sets
-//     the status word, and all roles drain and free TMEM before exiting.
+//     the status word, and all roles drain and free TMEM before exiting. Waiting
+//     threads let the hardware suspend them instead of polling shared memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
