@@ -45,7 +45,7 @@ def test_tiny_f32_workload_full():
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("T,F,C,h,d,H", [(7, 200, 2, 1, 128, 2), (5, 300, 3, 1, 64, 3), (4, 64, 1, 0, 128, 2),
-                                         (3, 130, 3, 0, 128, 1), (6, 1560, 3, 1, 128, 1)])
+                                         (3, 130, 3, 0, 128, 1), (6, 1560, 3, 1, 128, 1), (1, 100, 1, 0, 128, 1)])
 def test_window_small(dtype, T, F, C, h, d, H):
     w = wl.Workload("small", "window", 1, H, d, F, T, C, h, dtype=dtype, seed=T * 1000 + F)
     o, (q, k, v) = _bidir(w)
@@ -443,7 +443,7 @@ def test_full_lvsa_sampled():
     assert_parity("bf16", got, ref, "lvsa")
 
 
-@pytest.mark.parametrize("wf,stride,rot", [(3, 3, 1), (5, 4, 0), (1, 2, 3)])
+@pytest.mark.parametrize("wf,stride,rot", [(3, 3, 1), (5, 4, 0), (1, 2, 3), (3, 0, 0)])
 def test_lvsa_small(wf, stride, rot):
     w = wl.Workload("lvsa_small", "lvsa", 1, 2, 128, 300, 9, window_frames=wf, anchor_stride=stride,
                     rotation=rot, seed=37)
