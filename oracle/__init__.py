@@ -1,7 +1,7 @@
 """fp64 CPU oracle for hybrid softmax-window + linear-state attention.
 
 TEST INFRASTRUCTURE. Only the test suite, the package's smoke check and the
-benchmark's CPU-baseline leg import this package. The library never does, and
+benchmark's CPU-baseline and reference legs import this package. The library never does, and
 the oracle imports nothing from the library: the two share no code. Inputs come
 from the seeded generators, which contain none of the method's arithmetic.
 

@@ -33,7 +33,13 @@ the design notes):
     p the raster index inside the frame.
   * streaming: at step s the window is the chunks [s - n_win + 1, s]; older
     chunks are evicted into the linear set; window tiles the mask drops are
-    dropped (they reach neither branch).
+    dropped (they reach neither branch). With n_sink sink chunks, chunks
+    [0, n_sink) stay visible for good and the window starts no earlier than
+    n_sink; a denoising call of chunk s is the same computation with that
+    call's own K, V as chunk s.
+  * structured window + rotating anchors (Long Video Sparse Attention): keys
+    within (window_frames - 1) / 2 frames of the query, plus every key of an
+    anchor frame f with (f + rotation) % anchor_stride == 0.
 """
 from __future__ import annotations
 
