@@ -194,3 +194,33 @@ def test_stream_plan_with_sink(sink_frames):
         assert p["slots"] == [slot_of[c] for c in vis]
         assert len(set(p["slots"])) == len(vis)
         assert all(slot_of[c] == nwc + c for c in range(min(ns, s + 1)))
+
+
+def test_bench_work_counts_match_the_oracle_pair_counts():
+    """The effective FLOPs the bench reports come from the library layout; they must equal
+    4 d times the oracle's count of in-window (query, key) pairs plus the state FLOPs."""
+    import bench
+    w = wl.WAN13B_BIDIR
+    c = bench.work_counts(w)
+    pairs = oracle.effective_pairs_bidir(w.tokens_per_frame, w.n_frames, w.chunk_frames, w.halo_frames)
+    assert c["pairs_per_head"] == pairs
+    BH, d, N = w.B * w.H, w.d, w.N
+    assert c["total_flops"] == 4 * d * pairs * BH + BH * N * (2 * d * d + d) + BH * N * (2 * d * d + 2 * d)
+    # radial: pairs inside kept tiles, counted on the oracle's own mask
+    wr = wl.RADIAL_84F.with_(n_frames=12)
+    cr = bench.work_counts(wr)
+    tm = oracle.radial_tile_mask(wr.n_frames, wr.tokens_per_frame)[None]
+    assert cr["pairs_per_head"] == int(oracle.effective_pairs_tile_mask(tm, wr.N, wr.N)[0])
+
+
+def test_bench_stream_step_flops_by_brute_force():
+    import bench
+    w = wl.STREAM_HF
+    mask = wl.gen_stream_step(w, 5)[3]
+    flops, attn = bench.stream_step_flops(w, mask, True)
+    L, d, H = w.chunk_tokens, w.d, w.H
+    qlen = [min(128, L - 128 * i) for i in range(37)]
+    pairs = sum(int(mask[h, i, j]) * qlen[i] * qlen[j % 37] for h in range(H) for i in range(37)
+                for j in range(mask.shape[2]))
+    assert attn == 4 * d * pairs + H * L * (2 * d * d + 2 * d)
+    assert flops == attn + H * L * (2 * d * d + d)
