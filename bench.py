@@ -48,6 +48,9 @@ def parse():
     p.add_argument("--workload", default=wl.WAN13B_BIDIR.name, choices=sorted(wl.WORKLOADS))
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--schedule", choices=["pair", "single"], default="pair",
+                   help="tensor-core attention schedule of the bidirectional modes: a pair of query "
+                        "tiles per CTA (default) or one query tile per CTA (HYAT_FLAG_SINGLE_TILE)")
     return p.parse_args()
 
 
@@ -430,6 +433,7 @@ def main():
               **({"window_frames": w.window_frames, "anchor_stride": w.anchor_stride, "rotation": w.rotation}
                  if w.mode == "lvsa" else {}),
               "parallelism": f"replicas{world}" if world > 1 else "single",
+              "schedule": a.schedule,
               "l2": "inputs larger than L2 (Q,K,V,O %.0f MB > 126 MB); no flush" % (4 * w.B * w.H * w.N * w.d * 2 / 1e6)}
 
     if a.impl == "reference":
@@ -466,7 +470,9 @@ def main():
     q, k, v = wl.gen_qkv(w, seed=w.seed + rank)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     od = torch.empty_like(qd)
-    h = hyat.Hyat(hyat.config_from_workload(w), workload_mask(w), device=dev)
+    single = a.schedule == "single"
+    h = hyat.Hyat(hyat.config_from_workload(w, flags=hyat.FLAG_SINGLE_TILE if single else 0), workload_mask(w),
+                  device=dev)
     stream = torch.cuda.current_stream(dev)
     for _ in range(max(a.warmup, 3)):
         h.forward(qd, kd, vd, out=od)
@@ -498,6 +504,8 @@ def main():
     h.set_profiling(False)
     ms = max_over_ranks(ms, dev)
     launches = sum(n for _, n in kt.values())   # per-step launches x K (pass 2 mirrors pass 1)
+    if single:
+        launches += kt["attention"][1]          # each attention call is two kernels there (+ redo)
 
     value, tokens_per_s = job_throughput(counts["total_flops"], w.B * w.N, ms, world)
     pk, pk_src = peaks()
@@ -508,7 +516,7 @@ def main():
     if os.path.exists(tpath):
         t = json.load(open(tpath))
         sha = hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read() for f in KERNEL_SOURCES)).hexdigest()
-        if t.get("source_sha256") == sha and t.get("workload") == w.name:
+        if t.get("source_sha256") == sha and t.get("workload") == w.name and t.get("schedule", "pair") == a.schedule:
             traffic = t.get("dram_bytes_per_launch")
     roofline = {"bound": "tensor", "kernel": "attention", "achieved": achieved,
                 "timing": "per-launch CUDA events over a second pass of the same K steps",

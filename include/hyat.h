@@ -95,6 +95,13 @@ typedef enum {
  * 20 ms limit. The wait gives up, every role drains and frees TMEM, the status word is set,
  * and hyat_sync() returns HYAT_ERR_DEVICE_TIMEOUT; later calls on any handle work. */
 #define HYAT_FLAG_TEST_DEVICE_TIMEOUT 2u
+/* Schedule of the tensor-core attention in the bidirectional modes. By default a CTA runs a
+ * pair of query tiles, one per softmax warpgroup (the streaming mode always does). With this
+ * flag a CTA runs one query tile at a time: the two softmax warpgroups take alternate key
+ * tiles and TMEM holds three S buffers. Both schedules give results within the same
+ * tolerance; the second is currently the slower one on B200 and is kept for cross-checks and
+ * timing. */
+#define HYAT_FLAG_SINGLE_TILE 4u
 
 typedef struct {
   int32_t B, H, d;               /* d in {64, 128} */

@@ -23,7 +23,7 @@ int32_t nseg_pad64(int32_t n) { return (n + 63) / 64 * 64; }
 
 struct Plan {
   size_t status = 0, work = 0, entries = 0, pairs = 0, cm = 0, cm_bf16 = 0, sseg = 0, srest = 0, srest_bf16 = 0;
-  size_t ring_k = 0, ring_v = 0, mask = 0, fold_partial = 0, total = 0;
+  size_t ring_k = 0, ring_v = 0, mask = 0, fold_partial = 0, redo = 0, total = 0;
   int64_t n_work = 0, n_entries = 0;
 };
 
@@ -68,6 +68,7 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
     p.sseg = take(sizeof(float) * BH * L.nseg * E);
     p.srest = take(sizeof(float) * BH * L.nqg * E);
     p.srest_bf16 = take(2 * BH * L.nqg * c.d * c.d);
+    p.redo = take(sizeof(int4) * std::max<int64_t>(n_work, 1));
   }
   p.total = off;
   return p;
@@ -113,6 +114,12 @@ struct hyat_ctx {
   Entry* d_entries = nullptr;
   int4* d_pairs = nullptr;
   int32_t n_pairs = 0;
+  // one query tile per CTA (attn_single_kernel) with its redo list; the two counters live in
+  // the zeroed status region
+  bool single = false;
+  int4* d_redo = nullptr;
+  int32_t* d_redo_count = nullptr;
+  uint32_t* d_redo_done = nullptr;
   float* d_cm = nullptr;
   uint16_t* d_cm_bf16 = nullptr;
   bool use_gemm = false;             // tensor-core complement (block masks)
@@ -208,7 +215,11 @@ AttnArgs attn_args(hyat_ctx* h, const void* q, const void* k, const void* v, voi
 
 hyat_status launch_attention(hyat_ctx* h, const AttnArgs& a, cudaStream_t s) {
   cudaError_t e = timed(h, K_ATTN, s, [&] {
-    return h->use_tc ? launch_attn_tc(a, h->num_sms, s) : launch_attn_simt(a, s);
+    if (!h->use_tc) return launch_attn_simt(a, s);
+    if (!h->single) return launch_attn_tc(a, h->num_sms, s);
+    cudaError_t r = launch_attn_single(a, h->d_redo_count, h->d_redo, h->num_sms, s);
+    if (r == cudaSuccess) r = launch_attn_tc_redo(a, h->d_redo, h->d_redo_count, h->d_redo_done, h->num_sms, s);
+    return r;
   });
   if (e != cudaSuccess) return cuda_fail(h, e, "attention kernel");
   return HYAT_OK;
@@ -287,7 +298,10 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
     h->d_cm = reinterpret_cast<float*>(ws + h->plan.cm);
     if (h->plan.cm_bf16) h->d_cm_bf16 = reinterpret_cast<uint16_t*>(ws + h->plan.cm_bf16);
     h->d_sseg = reinterpret_cast<float*>(ws + h->plan.sseg);
+    h->d_redo = reinterpret_cast<int4*>(ws + h->plan.redo);
   }
+  h->d_redo_count = reinterpret_cast<int32_t*>(ws + h->plan.status + 64);
+  h->d_redo_done = reinterpret_cast<uint32_t*>(ws + h->plan.status + 128);
 
   int dev = 0, major = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -321,6 +335,9 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
     const int32_t nqt = tiles(stream_chunk_tokens(*cfg));
     pairs = build_stream_pairs(h->BH, nqt);
     if (prefer_split_pairs(pairs.size(), h->num_sms)) pairs = build_split_pairs(size_t(h->BH) * nqt);
+  } else if (h->use_tc && (cfg->flags & HYAT_FLAG_SINGLE_TILE)) {
+    pairs = build_single_items(h->lay.work, h->num_sms);
+    h->single = true;
   } else {
     pairs = choose_pairs(h->lay.work, h->num_sms);
   }

@@ -76,6 +76,7 @@ struct __align__(1024) Smem {
   int32_t abort_flag;
   uint64_t never;                // test hook: a barrier nothing arrives on
   unsigned long long timeout_ns; // limit of every bounded wait
+  int32_t n_pairs;               // pairs of this launch (read on the device in redo mode)
 };
 
 struct TcParams {
@@ -91,6 +92,10 @@ struct TcParams {
   uint32_t* status;
   int32_t test_timeout;    // test hook: wait once on a barrier nothing signals (20 ms limit)
   int32_t phi;             // feature map of the linear branch (hyat_phi)
+  // Redo mode: the pair count is read on the device from *n_pairs_dev (written by the kernel
+  // before this one), and the last CTA to finish resets it and *done_count to 0.
+  int32_t* n_pairs_dev;
+  uint32_t* done_count;
 };
 
 // Bounded wait on a phase parity. Returns false if the kernel is aborting. After the first
@@ -200,7 +205,8 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
   uint32_t qph = 0, sph = 0, xph = 0;
   uint32_t pv_phase = 0;                            // pv_done phases completed before this pair
   bool o1_busy = false;                             // slot 1: O1 not yet read out by slot 0
-  for (int pi = blockIdx.x; pi < p.n_pairs; pi += gridDim.x) {
+  const int n_pairs = sm->n_pairs;
+  for (int pi = blockIdx.x; pi < n_pairs; pi += gridDim.x) {
     const PairView pv = pair_view(p, pi);
     if (s == 1 && !pv.has1) continue;
     const WorkItem wi = p.work[s == 0 ? pv.item[0] : pv.item[1]];
@@ -367,6 +373,20 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
   }
 }
 
+// Redo mode: every CTA has read the pair count by the time it gets here; the last one to
+// arrive resets the count and this counter for the next launch.
+__device__ __forceinline__ void redo_finish(const TcParams& p) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.done_count, 1u) == gridDim.x - 1) {
+      *reinterpret_cast<volatile int32_t*>(p.n_pairs_dev) = 0;
+      *reinterpret_cast<volatile uint32_t*>(p.done_count) = 0u;
+      __threadfence();
+    }
+  }
+}
+
 // ------------------------------------------------------------------ the kernel
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -375,6 +395,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   Smem* sm = reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n_pairs = p.n_pairs;
+  if (p.n_pairs_dev) {
+    // redo mode: the count comes from the kernel before this one; CTAs without work leave
+    // before they allocate anything
+    pdl_wait();
+    n_pairs = *reinterpret_cast<volatile const int32_t*>(p.n_pairs_dev);
+    if (static_cast<int>(blockIdx.x) >= n_pairs) {
+      redo_finish(p);
+      return;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
@@ -394,6 +425,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&sm->never, 1);
     sm->abort_flag = 0;
     sm->timeout_ns = p.test_timeout ? 20000000ull : kTimeoutNs;
+    sm->n_pairs = n_pairs;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -424,7 +456,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (++st == NS) { st = 0; ph ^= 1u; }
         return true;
       };
-      for (int pi = blockIdx.x; pi < p.n_pairs && ok; pi += gridDim.x) {
+      for (int pi = blockIdx.x; pi < sm->n_pairs && ok; pi += gridDim.x) {
         const PairView pv = pair_view(p, pi);
         const bool has1 = pv.has1, shared = pv.shared;
         const WorkItem w0 = p.work[pv.item[0]];
@@ -516,7 +548,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit_elect(done);
       };
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
-      for (int pi = blockIdx.x; pi < p.n_pairs && ok; pi += gridDim.x) {
+      for (int pi = blockIdx.x; pi < sm->n_pairs && ok; pi += gridDim.x) {
         const PairView pvw = pair_view(p, pi);
         const bool has1 = pvw.has1, shared = pvw.shared, split = pvw.split;
         const int n0 = pvw.n[0], n1 = pvw.n[1];
@@ -611,6 +643,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == MMA_WARP) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
+  if (p.n_pairs_dev) redo_finish(p);
 }
 
 // ------------------------------------------------------------------ host side
@@ -621,7 +654,8 @@ static_assert(kSmemBytes <= 232448, "shared memory above the 227 KB a CTA can ha
 
 bool attn_tc_supported(int d, int dtype) { return d == D && dtype == HYAT_BF16; }
 
-cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s) {
+static cudaError_t launch_attn_tc_impl(const AttnArgs& a, int32_t* n_pairs_dev, uint32_t* done_count, int num_sms,
+                               cudaStream_t s) {
   if (a.n_pairs == 0) return cudaSuccess;
   CUtensorMap mq, mk, mv, ms;       // 128-row boxes: two loads of 64 x 128 bf16 = TILE_BYTES
   static_assert(2 * 64 * 128 * 2 == TILE_BYTES, "tile bytes must match the two TMA boxes");
@@ -648,8 +682,22 @@ cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s) {
   p.status = a.status;
   p.test_timeout = a.test_timeout;
   p.phi = a.phi;
+  p.n_pairs_dev = n_pairs_dev;
+  p.done_count = done_count;
   const int grid = a.n_pairs < num_sms ? a.n_pairs : num_sms;
   return launch_pdl(attn_tc_kernel, dim3(grid), dim3(NUM_THREADS), kSmemBytes, s, mq, mk, mv, ms, p);
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s) {
+  return launch_attn_tc_impl(a, nullptr, nullptr, num_sms, s);
+}
+
+cudaError_t launch_attn_tc_redo(const AttnArgs& a, const int4* redo_items, int32_t* redo_count,
+                                uint32_t* done_count, int num_sms, cudaStream_t s) {
+  AttnArgs r = a;
+  r.pairs = redo_items;
+  r.n_pairs = a.n_pairs < num_sms ? a.n_pairs : num_sms;   // grid; the count is read on the device
+  return launch_attn_tc_impl(r, redo_count, done_count, num_sms, s);
 }
 
 }  // namespace hyat

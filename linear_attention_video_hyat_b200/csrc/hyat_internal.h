@@ -161,6 +161,15 @@ struct AttnArgs {
 };
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s);
+// One query tile per CTA at a time (a.pairs = {item, -1, 0, 0} in processing order, a.n_pairs
+// of them). Tiles whose row sums leave the safe range are appended to redo_items (count at
+// *redo_count, at most a.n_pairs); launch_attn_tc_redo then recomputes them with
+// attn_tc_kernel, reading the count on the device and resetting it (and *done_count) to 0.
+cudaError_t launch_attn_single(const AttnArgs& a, int32_t* redo_count, int4* redo_items, int num_sms,
+                               cudaStream_t s);
+cudaError_t launch_attn_tc_redo(const AttnArgs& a, const int4* redo_items, int32_t* redo_count,
+                                uint32_t* done_count, int num_sms, cudaStream_t s);
+std::vector<int4> build_single_items(const std::vector<WorkItem>& work, int32_t num_sms);
 bool attn_tc_supported(int d, int dtype);
 
 struct RingCopyArgs {

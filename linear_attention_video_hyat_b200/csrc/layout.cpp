@@ -296,6 +296,12 @@ std::vector<int4> choose_pairs(const std::vector<WorkItem>& work, int32_t num_sm
   return order_pairs_for_grid(pairs, work, num_sms);
 }
 
+std::vector<int4> build_single_items(const std::vector<WorkItem>& work, int32_t num_sms) {
+  std::vector<int4> items(work.size());
+  for (size_t i = 0; i < work.size(); ++i) items[i] = make_int4(static_cast<int>(i), -1, 0, 0);
+  return order_pairs_for_grid(items, work, num_sms);
+}
+
 std::vector<int4> build_stream_pairs(int32_t BH, int32_t nqt) {
   std::vector<int4> pairs;
   for (int32_t bh = 0; bh < BH; ++bh)

@@ -22,6 +22,7 @@ F32, BF16 = 0, 1
 MODE_WINDOW, MODE_BLOCKMASK, MODE_RADIAL, MODE_STREAM = range(4)
 FLAG_SIMT = 1
 FLAG_TEST_DEVICE_TIMEOUT = 2
+FLAG_SINGLE_TILE = 4
 TILE = 128
 KERNEL_KINDS = ("state", "complement", "attention", "fold_ring", "layout_prep")
 

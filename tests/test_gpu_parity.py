@@ -396,11 +396,11 @@ def _lvsa_masks(w):
     return lib_mask[None], ref_mask[None]
 
 
-def _bidir_sampled(w, heads, per_tile=2, seed=0):
+def _bidir_sampled(w, heads, per_tile=2, seed=0, flags=0):
     lib_mask = ref_mask = None
     if w.mode == "lvsa":
         lib_mask, ref_mask = _lvsa_masks(w)
-    o, (q, k, v) = _bidir(w, mask=lib_mask)
+    o, (q, k, v) = _bidir(w, mask=lib_mask, flags=flags)
     N = w.N
     if w.mode == "window":
         C = w.chunk_tokens
@@ -462,3 +462,89 @@ def test_full_stream_sampled():
     for s, (got, ref) in outs.items():
         assert_parity("bf16", got, ref, f"step {s}")
     h.close()
+
+
+# ------------------------------------------------------------------ single-tile schedule
+# HYAT_FLAG_SINGLE_TILE: one query tile per CTA, two softmax warpgroups on alternate key
+# tiles, three S buffers, fixed reference max with a redo list for tiles out of range.
+SINGLE = hyat.FLAG_SINGLE_TILE
+
+
+@pytest.mark.parametrize("T,F,C,h,H", [(7, 200, 2, 1, 2), (4, 64, 1, 0, 2), (3, 130, 3, 0, 1), (6, 1560, 3, 1, 1),
+                                       (1, 100, 1, 0, 1), (3, 100, 1, 1, 1), (5, 100, 2, 1, 1), (8, 100, 4, 1, 1)])
+def test_single_tile_window_small(T, F, C, h, H):
+    """Query tiles of 1 to 61 key tiles: every count of S-buffer fills mod 3 and both warpgroups
+    with no tile at all (a query tile with one key tile leaves warpgroup 1 only the linear term)."""
+    w = wl.Workload("single", "window", 1, H, 128, F, T, C, h, seed=T * 100 + F)
+    o, (q, k, v) = _bidir(w, flags=SINGLE)
+    assert_parity("bf16", f64(o), _window_ref(w, q, k, v), (T, F, C, h, H))
+
+
+@pytest.mark.parametrize("sigma", [6.0, 20.0])
+def test_single_tile_large_logits_take_the_redo_list(sigma):
+    """Row sums beyond 2^100 under the fixed reference max: those query tiles are recomputed by
+    the pair kernel, which moves its reference max; the result must be as exact as there."""
+    w = wl.Workload("large_logits", "window", 1, 2, 128, 300, 4, 2, 1, seed=17)
+    q, k, v = wl.gen_qkv(w)
+    q = (q.float() * sigma).to(torch.bfloat16)
+    k = (k.float() * sigma).to(torch.bfloat16)
+    h = hyat.Hyat(hyat.config_from_workload(w, flags=SINGLE))
+    for rep in range(2):            # the second call finds the redo list emptied by the first
+        o = h.forward(*_dev(q, k, v))
+        h.sync()
+        assert_bf16_peaked(f64(o.cpu()), _window_ref(w, q, k, v), f64(v), sigma)
+    # and a unit-scale call on the same handle after that is exact too
+    q2, k2, v2 = wl.gen_qkv(w.with_(seed=18))
+    o2 = h.forward(*_dev(q2, k2, v2))
+    h.sync()
+    assert_parity("bf16", f64(o2.cpu()), _window_ref(w, q2, k2, v2), "after redo")
+    h.close()
+
+
+@pytest.mark.parametrize("kind", ["random", "zeros", "ones"])
+def test_single_tile_blockmask(kind):
+    T, F, H = 5, 230, 2
+    nT = -(-T * F // 128)
+    mask = {"random": wl.gen_tile_mask(H, nT, nT, seed=4),
+            "zeros": np.zeros((H, nT, nT), np.uint8),
+            "ones": np.ones((H, nT, nT), np.uint8)}[kind]
+    w = wl.Workload("bm", "blockmask", 1, H, 128, F, T, seed=5)
+    o, (q, k, v) = _bidir(w, mask=mask, mask_heads=H, flags=SINGLE)
+    assert_parity("bf16", f64(o), oracle.blockmask_attention(f64(q), f64(k), f64(v), mask), kind)
+
+
+@pytest.mark.parametrize("phi", ["relu", "exp"])
+def test_single_tile_feature_maps(phi):
+    w = wl.Workload("single_phi", "window", 1, 2, 128, 200, 7, 2, 1, seed=8, phi=phi)
+    o, (q, k, v) = _bidir(w, flags=SINGLE)
+    ref = oracle.bidir_window_attention(f64(q), f64(k), f64(v), 200, 7, 2, 1, phi=phi)
+    assert_parity("bf16", f64(o), ref, phi)
+
+
+def test_single_tile_radial_and_lvsa_small():
+    w = wl.Workload("radial_small", "radial", 1, 2, 128, 300, 9, seed=6)
+    o, (q, k, v) = _bidir(w, flags=SINGLE)
+    assert_parity("bf16", f64(o), oracle.radial_attention(f64(q), f64(k), f64(v), 9, 300), "radial")
+    w = wl.Workload("lvsa_small", "lvsa", 1, 2, 128, 300, 9, window_frames=3, anchor_stride=3, rotation=1, seed=37)
+    lib_mask, ref_mask = _lvsa_masks(w)
+    o, (q, k, v) = _bidir(w, mask=lib_mask, flags=SINGLE)
+    assert_parity("bf16", f64(o), oracle.blockmask_attention(f64(q), f64(k), f64(v), ref_mask), "lvsa")
+
+
+def test_single_tile_device_timeout_is_reported_and_recoverable():
+    w = wl.Workload("timeout", "window", 1, 2, 128, 200, 4, 2, 1, seed=2)
+    q, k, v = _dev(*wl.gen_qkv(w))
+    h = hyat.Hyat(hyat.config_from_workload(w, flags=SINGLE | hyat.FLAG_TEST_DEVICE_TIMEOUT))
+    h.forward(q, k, v)
+    with pytest.raises(hyat.HyatError) as ei:
+        h.sync()
+    assert ei.value.status == hyat.ERR_DEVICE_TIMEOUT
+    h.close()
+    o, _ = _bidir(w, flags=SINGLE, qkv=tuple(t.cpu() for t in (q, k, v)))
+    assert_parity("bf16", f64(o), _window_ref(w, *(t.cpu() for t in (q, k, v))), "after a device timeout")
+
+
+@pytest.mark.slow
+def test_single_tile_full_wan13b_sampled():
+    got, ref = _bidir_sampled(wl.WAN13B_BIDIR, heads=[0, 5, 11], flags=SINGLE)
+    assert_parity("bf16", got, ref, "wan1.3b single tile")
