@@ -33,3 +33,4 @@ from .hybrid import (  # noqa: F401
     effective_pairs_bidir,
     effective_pairs_tile_mask,
 )
+from .rope import temporal_offsets, rope_temporal  # noqa: F401,E402

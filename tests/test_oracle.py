@@ -413,3 +413,45 @@ def test_lvsa_tile_mask_invariants():
     win = oracle.lvsa_tile_mask(T, F, 3, 0, 0, tile=16)                                    # no anchors: banded
     assert np.all(win == win.T)
     assert base.sum() > win.sum()
+
+
+# ------------------------------------------------------------------ capped temporal RoPE
+# Pins for oracle.rope_temporal from the mathematics of rotations, independent of its code.
+def test_rope_complex_form_and_identities():
+    """Pair i of a token of offset p, read as the complex number x[2i] + i x[2i+1], is
+    multiplied by exp(i p theta_i); the band's width 0 and offset 0 leave x unchanged."""
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((2, 30, 16))
+    F, f0, ref, cap, t, base = 4, 3, 1, 5, 10, 100.0
+    got = oracle.rope_temporal(x, F, f0, ref, cap, t, base)
+    p = np.minimum(f0 + np.arange(30) // F - ref, cap - 1)
+    z = x[..., 0::2] + 1j * x[..., 1::2]
+    theta = np.array([base ** (-2.0 * i / t) if i < t // 2 else 0.0 for i in range(8)])
+    zr = z * np.exp(1j * p[:, None] * theta[None, :])
+    want = np.empty_like(x)
+    want[..., 0::2], want[..., 1::2] = zr.real, zr.imag
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(oracle.rope_temporal(x, F, f0, ref, cap, 0, base), x)
+    same = oracle.rope_temporal(x, F, ref, ref, cap, t, base)[:, :F]      # first frame: p = 0
+    np.testing.assert_array_equal(same, x[:, :F])
+
+
+def test_rope_is_relative_and_capped():
+    """Inside the cap, q at offset a against k at offset b depends on a - b only; norms are
+    kept; beyond the cap every frame turns like offset cap - 1."""
+    rng = np.random.default_rng(42)
+    d, t, F, cap = 8, 8, 1, 6
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    x = np.stack([q, k])[:, None, :].repeat(10, axis=1)                   # tokens = frames 0..9
+    rq = oracle.rope_temporal(x[0], F, 0, 0, cap, t)
+    rk = oracle.rope_temporal(x[1], F, 0, 0, cap, t)
+    for a, b, a2, b2 in [(3, 1, 4, 2), (5, 5, 0, 0), (2, 4, 0, 2)]:
+        assert abs(rq[a] @ rk[b] - rq[a2] @ rk[b2]) < 1e-12
+    np.testing.assert_allclose(np.linalg.norm(rq, axis=1), np.linalg.norm(q), rtol=1e-13)
+    for f in range(cap, 10):
+        np.testing.assert_array_equal(rq[f], rq[cap - 1])
+    assert np.abs(rq[cap - 1] - rq[cap - 2]).max() > 1e-3
+    with pytest.raises(ValueError):
+        oracle.rope_temporal(x[0], F, 0, 1, cap, t)                        # frame before the reference
+    with pytest.raises(ValueError):
+        oracle.rope_temporal(x[0], F, 0, 0, cap, 7)                        # odd band
