@@ -37,6 +37,9 @@ METRIC = "hybrid-attn effective TFLOP/s & tokens/s per layer; % of B200 BF16 TC 
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["linear_attention_video_hyat_b200/csrc/attn_tc.cu"]
+# the streaming bench's --rope step: a temporal band of 44 of the 128 head dimensions, the
+# index capped at 21 frames (the pages' example of a pretrained model's range), base 10000
+ROPE = {"t_dims": 44, "cap": 21, "base": 10000.0}
 
 
 def parse():
@@ -51,6 +54,9 @@ def parse():
     p.add_argument("--schedule", choices=["pair", "single"], default="pair",
                    help="tensor-core attention schedule of the bidirectional modes: a pair of query "
                         "tiles per CTA (default) or one query tile per CTA (HYAT_FLAG_SINGLE_TILE)")
+    p.add_argument("--rope", action="store_true",
+                   help="streaming workload: each step first applies the capped temporal RoPE "
+                        "(hyat_rope_temporal) to the chunk's Q and K")
     return p.parse_args()
 
 
@@ -281,6 +287,8 @@ def bench_stream(a, w, rank, world, local):
               "window_frames": w.window_frames, "mode": w.mode, "mask": "Bernoulli(0.5) + diagonal tiles",
               "parallelism": f"replicas{world}" if world > 1 else "single",
               "l2": "per step: fresh Q, K, V (86 MB) and the ring (86 MB); no flush"}
+    if a.rope:
+        config["rope"] = dict(ROPE, ref="first frame of the oldest window chunk")
     n_dist = 4           # distinct steady-state inputs, cycled
     inputs = [wl.gen_stream_step(w, nwc + i, seed=w.seed + rank) for i in range(n_dist)]
     flops = [stream_step_flops(w, m, True) for _, _, _, m in inputs]
@@ -329,12 +337,33 @@ def bench_stream(a, w, rank, world, local):
     od = torch.empty_like(dev_in[0][0])
     stream = torch.cuda.current_stream(dev)
 
-    def run(h, steps, first):
+    n_sink = w.sink_frames // w.chunk_frames
+    qr, kr = torch.empty_like(od), torch.empty_like(od)
+    rope_events = []
+
+    def rope(q, k, s, timed=False):
+        """The step before attention: Q and K of chunk s turned by their capped offsets from
+        the oldest window chunk's first frame."""
+        f0 = s * w.chunk_frames
+        ref = max(n_sink, s - nwc + 1) * w.chunk_frames
+        if timed:
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[0].record(stream)
+        for x, y in ((q, qr), (k, kr)):
+            hyat.rope_temporal(x, w.tokens_per_frame, f0, ref, ROPE["cap"], ROPE["t_dims"], ROPE["base"], out=y)
+        if timed:
+            ev[1].record(stream)
+            rope_events.append(ev)
+        return qr, kr
+
+    def run(h, steps, first, timed=False):
         for i in range(steps):
             s = first + i
             q, k, v, m = dev_in[s % n_dist]
             if s < nwc:       # the window is still filling: masks of the growing shape
                 m = wl.gen_stream_step(w, s, seed=w.seed + rank)[3]
+            if a.rope:
+                q, k = rope(q, k, s, timed)
             h.stream_step(q, k, v, mask=m, out=od)
 
     h = hyat.Hyat(cfg, device=dev)
@@ -354,11 +383,11 @@ def bench_stream(a, w, rank, world, local):
     h.set_profiling(True)
     h.kernel_times()
     with ClockSampler(local) as clk2:
-        run(h, a.steps, warm + a.steps)
+        run(h, a.steps, warm + a.steps, timed=True)
         torch.cuda.synchronize(dev)
     kt = h.kernel_times()
     h.set_profiling(False)
-    launches = sum(n for _, n in kt.values())
+    launches = sum(n for _, n in kt.values()) + 2 * len(rope_events)
     value, tokens_per_s = job_throughput(mean_flops, w.B * w.chunk_tokens, ms, world)
     pk, pk_src = peaks()
     attn_ms = kt["attention"][0] / max(kt["attention"][1], 1)
@@ -371,6 +400,12 @@ def bench_stream(a, w, rank, world, local):
                 "frac_sustained": achieved / pk["bf16_tflops_sustained"], "traffic": None,
                 "launch_ms": attn_ms, "algorithmic_flops_per_launch": mean_attn}
     kernels = {k_: {"ms_per_launch": t_ / max(n_, 1), "launches": n_} for k_, (t_, n_) in kt.items() if n_}
+    if rope_events:
+        r_ms = sum(e0.elapsed_time(e1) for e0, e1 in rope_events) / (2 * len(rope_events))
+        r_bytes = 2 * od.numel() * od.element_size()        # out of place: one read, one write
+        kernels["rope"] = {"ms_per_launch": r_ms, "launches": 2 * len(rope_events),
+                           "hbm_gbs": r_bytes / (r_ms / 1e3) / 1e9,
+                           "timing": "CUDA events around the Q and K calls of each step, pass 2"}
 
     e2e = None
     if not a.no_e2e:
@@ -383,7 +418,8 @@ def bench_stream(a, w, rank, world, local):
             for i in range(steps):
                 qh, kh_, vh, m = pinned[(first + i) % n_dist]
                 qd.copy_(qh, non_blocking=True); kd.copy_(kh_, non_blocking=True); vd.copy_(vh, non_blocking=True)
-                h.stream_step(qd, kd, vd, mask=m, out=od)
+                qx, kx = rope(qd, kd, warm + 2 * a.steps + first + i) if a.rope else (qd, kd)
+                h.stream_step(qx, kx, vd, mask=m, out=od)
                 oh.copy_(od, non_blocking=True)
         run_e2e(0, 2)
         torch.cuda.synchronize(dev)

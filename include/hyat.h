@@ -249,6 +249,31 @@ HYAT_API hyat_status hyat_kernel_times(hyat_handle h, double* ms, int64_t* launc
 HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, const void* q, const void* k,
                                             const void* v, void* o, void* stream);
 
+/* ---- the step before attention ---- */
+
+/* Temporal rotary position embedding with a capped relative index (Long-Horizon Streaming
+ * Video Generation via Hybrid Attention with Decoupled Distillation, Section 2.C, the relative
+ * RoPE constraint: the temporal RoPE index is written relative to a reference frame and held
+ * below an upper bound, so that generation of any length stays inside the index range the
+ * pretrained model has seen). The pages give no formula; this reading applies rotary pairs in
+ * their usual form to the first t_dims dimensions of each head:
+ *   (x[2i], x[2i+1]) turns by the angle p * base^(-2i / t_dims) for i < t_dims / 2,
+ *   p = min(frame - ref_frame, cap - 1),  frame = first_frame + token / tokens_per_frame,
+ * and leaves dimensions t_dims .. d-1 unchanged (a 3-D embedding rotates them by spatial
+ * position, which the cap does not concern). Apply it to Q and K before the attention call.
+ *   x, y    device tensors [BH, n_tokens, d] of dtype (HYAT_F32 or HYAT_BF16), 16-byte
+ *           aligned, owned by the caller; y == x works in place (then only the band is
+ *           rewritten), other overlaps are not allowed;
+ *   d       64 or 128; t_dims even, 0 <= t_dims <= d; cap >= 1; base > 0 and finite;
+ *           first_frame >= ref_frame; BH <= 65535.
+ * Angles and their sines and cosines are formed in double, the rotation in fp32. Enqueued
+ * on `stream`; returns HYAT_ERR_INVALID_ARG (nothing enqueued) on bad arguments and
+ * HYAT_ERR_CUDA if the launch fails. BH or n_tokens 0 is a no-op. */
+HYAT_API hyat_status hyat_rope_temporal(const void* x, void* y, int32_t BH, int32_t n_tokens, int32_t d,
+                                        int32_t dtype, int32_t tokens_per_frame, int32_t first_frame,
+                                        int32_t ref_frame, int32_t cap, int32_t t_dims, float base,
+                                        void* stream);
+
 #ifdef __cplusplus
 }
 #endif

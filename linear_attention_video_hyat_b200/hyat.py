@@ -34,7 +34,7 @@ EXPORTED = (
     "hyat_destroy", "hyat_last_error", "hyat_status_string", "hyat_plan_layout", "hyat_radial_mask",
     "hyat_stream_plan", "hyat_stream_state_bytes", "hyat_stream_get_state", "hyat_stream_set_state",
     "hyat_set_profiling", "hyat_kernel_times", "hyat_fwd_bidir_noalloc", "hyat_fwd_stream_denoise",
-    "hyat_lvsa_mask",
+    "hyat_lvsa_mask", "hyat_rope_temporal",
 )
 
 
@@ -82,6 +82,7 @@ def _load():
         "hyat_set_profiling": (ctypes.c_int, [P, ctypes.c_int]),
         "hyat_kernel_times": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I64), ctypes.c_int]),
         "hyat_fwd_bidir_noalloc": (ctypes.c_int, [CP, P, P, P, P, P]),
+        "hyat_rope_temporal": (ctypes.c_int, [P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, ctypes.c_float, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -147,6 +148,24 @@ def lvsa_mask(n_frames: int, tokens_per_frame: int, window_frames: int, anchor_s
     out = np.zeros((nT, nT), np.uint8)
     _check(lib.hyat_lvsa_mask(n_frames, tokens_per_frame, window_frames, anchor_stride, rotation,
                               out.ctypes.data, out.size))
+    return out
+
+
+def rope_temporal(x, tokens_per_frame: int, first_frame: int, ref_frame: int, cap: int, t_dims: int,
+                  base: float = 10000.0, out=None, stream=None):
+    """Capped relative temporal RoPE (see hyat_rope_temporal) of a contiguous CUDA tensor
+    [..., n_tokens, d] (f32 or bf16); out=x works in place."""
+    dt = {torch.float32: F32, torch.bfloat16: BF16}.get(x.dtype)
+    if x.device.type != "cuda" or dt is None or not x.is_contiguous() or x.dim() < 2:
+        raise ValueError("need a contiguous f32 or bf16 CUDA tensor [..., n_tokens, d]")
+    out = torch.empty_like(x) if out is None else out
+    if out.shape != x.shape or out.dtype != x.dtype or not out.is_contiguous() or out.device != x.device:
+        raise ValueError("out must match x")
+    n, d = x.shape[-2], x.shape[-1]
+    bh = x.numel() // max(n * d, 1) if n * d else 0
+    s = torch.cuda.current_stream(x.device) if stream is None else stream
+    _check(lib.hyat_rope_temporal(x.data_ptr(), out.data_ptr(), bh, n, d, dt, tokens_per_frame, first_frame,
+                                  ref_frame, cap, t_dims, float(base), s.cuda_stream))
     return out
 
 

@@ -224,3 +224,18 @@ def test_bench_stream_step_flops_by_brute_force():
                 for j in range(mask.shape[2]))
     assert attn == 4 * d * pairs + H * L * (2 * d * d + 2 * d)
     assert flops == attn + H * L * (2 * d * d + d)
+
+
+def test_rope_temporal_validates_before_touching_the_gpu():
+    """Bad arguments return HYAT_ERR_INVALID_ARG and empty tensors are a no-op, with no launch."""
+    f = hyat.lib.hyat_rope_temporal
+    good = dict(BH=2, n=10, d=128, dt=hyat.BF16, F=5, f0=3, ref=1, cap=4, t=44, base=10000.0)
+
+    def call(x=None, y=None, **kw):
+        a = dict(good, **kw)
+        return f(x, y, a["BH"], a["n"], a["d"], a["dt"], a["F"], a["f0"], a["ref"], a["cap"], a["t"], a["base"], None)
+    assert call(BH=0) == hyat.OK and call(n=0) == hyat.OK
+    assert call() == hyat.ERR_INVALID_ARG                                      # null tensors
+    for bad in (dict(d=96), dict(dt=7), dict(F=0), dict(cap=0), dict(t=45), dict(t=130), dict(t=-2),
+                dict(base=0.0), dict(base=float("inf")), dict(f0=0, ref=1), dict(BH=-1), dict(BH=70000)):
+        assert call(**bad) == hyat.ERR_INVALID_ARG, bad
