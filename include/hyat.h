@@ -245,7 +245,8 @@ HYAT_API hyat_status hyat_kernel_times(hyat_handle h, double* ms, int64_t* launc
  * leaves the previous call's contents in it (the status word is cleared on
  * each call): calls that overlap on the GPU -- on different streams, or from
  * different threads -- race on it and must be serialised by the caller.
- * Device-side timeouts of this path are not reported (there is no handle). */
+ * Device-side timeouts of this path are not reported (there is no handle). The attention
+ * always runs the pair schedule (HYAT_FLAG_SINGLE_TILE is ignored here). */
 HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, const void* q, const void* k,
                                             const void* v, void* o, void* stream);
 
