@@ -86,27 +86,12 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// K-major operand (rows = M or N, 128 columns of K in two 64-column halves); K step kk of 16
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int kk) {
-  return sdesc(base + (kk >> 2) * HALF_BYTES + (kk & 3) * 32, 16, 1024);
-}
-// MN-major operand (rows = K, 128 columns of N in two 64-column halves); K step kk of 16 rows
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int kk) {
-  return sdesc(base + kk * 2048, HALF_BYTES, 1024);
-}
 
 __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
 }
 
 // Warp-wide forms: every lane of a converged warp executes the instruction and elect.sync
