@@ -219,6 +219,49 @@ def cpu_threads():
         return os.cpu_count()
 
 
+def cpu_info():
+    """The host the oracle runs on: CPU model, logical cores, and the BLAS library with its
+    thread count (the oracle's matrix products run in it)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    blas = None
+    try:
+        import threadpoolctl
+        for i in threadpoolctl.threadpool_info():
+            if i.get("user_api") == "blas":
+                blas = {"library": i.get("internal_api"), "threads": i.get("num_threads")}
+                break
+    except Exception:
+        pass
+    return {"cpu_model": model, "logical_cores": os.cpu_count(), "blas": blas}
+
+
+def oracle_work_counts(w):
+    """Effective FLOPs of one call from the oracle's own window and mask rules (the reference
+    arm never loads the library)."""
+    import oracle
+    if w.mode == "window":
+        pairs = int(oracle.effective_pairs_bidir(w.tokens_per_frame, w.n_frames, w.chunk_frames, w.halo_frames))
+    else:
+        if w.mode == "radial":
+            tm = oracle.radial_tile_mask(w.n_frames, w.tokens_per_frame)[None]
+        else:
+            tm = oracle.lvsa_tile_mask(w.n_frames, w.tokens_per_frame, w.window_frames, w.anchor_stride,
+                                       w.rotation)[None]
+        pairs = int(oracle.effective_pairs_tile_mask(tm, w.N, w.N)[0])
+    BH, d, N = w.B * w.H, w.d, w.N
+    soft = 4 * d * pairs * BH
+    state = BH * N * (2 * d * d + d) + BH * N * (2 * d * d + 2 * d)
+    return {"pairs_per_head": pairs, "total_flops": soft + state}
+
+
 def cpu_rate(w, counts, n_blocks, qkv=None):
     secs, rows = oracle_sample(w, n_blocks, qkv=qkv)
     total_rows = w.B * w.H * w.N
@@ -329,7 +372,8 @@ def bench_stream(a, w, rank, world, local):
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
                 "impl": "reference", "tokens_per_s": rows_done / secs,
                 "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-                                 "sample": f"{a.steps} blocks of 256 query rows (one head each) of a steady step"},
+                                 "sample": f"{a.steps} blocks of 256 query rows (one head each) of a steady step",
+                                 **cpu_info()},
                 "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
@@ -470,7 +514,6 @@ def main():
     if w.mode == "stream":
         return bench_stream(a, w, rank, world, local)
     assert w.mode in ("window", "radial", "lvsa"), "the bench times a bidirectional layer call or streaming steps"
-    counts = work_counts(w)
     config = {"workload": w.name, "B": w.B, "H": w.H, "d": w.d, "tokens": w.N,
               "tokens_per_frame": w.tokens_per_frame, "frames": w.n_frames, "mode": w.mode,
               "chunk_frames": w.chunk_frames, "halo_frames": w.halo_frames,
@@ -483,6 +526,7 @@ def main():
     if a.impl == "reference":
         if rank != 0:
             return 0
+        counts = oracle_work_counts(w)
         qkv = wl.gen_qkv(w)
         for _ in range(a.warmup):
             oracle_sample(w, 1, seed=99, qkv=qkv)
@@ -498,12 +542,14 @@ def main():
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
                 "impl": "reference", "tokens_per_s": rows / secs,
                 "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-                                 "sample": f"{a.steps} blocks of 256 query rows (one head each) per run"},
+                                 "sample": f"{a.steps} blocks of 256 query rows (one head each) per run",
+                                 **cpu_info()},
                 "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
 
     from linear_attention_video_hyat_b200 import hyat
+    counts = work_counts(w)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -597,7 +643,7 @@ def main():
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         tf, rps, secs, rows = cpu_rate(w, counts, n_blocks=24, qkv=(q, k, v))
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
-               "tokens_per_s": rps, "seconds": secs,
+               "tokens_per_s": rps, "seconds": secs, **cpu_info(),
                "sample": f"{rows} query rows (24 blocks of 256 rows, one head each) of the same layer; "
                          f"FLOPs scaled by the sampled fraction of rows"}
 

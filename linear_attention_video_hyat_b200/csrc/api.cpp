@@ -523,7 +523,9 @@ hyat_status hyat_sync(hyat_handle h) {
   e = cudaMemcpy(&status, h->d_status, sizeof(status), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(h, e, "status read");
   if (status) {
-    cudaMemset(h->d_status, 0, sizeof(status));
+    // The status region also holds the single-tile schedule's redo count and its finish
+    // counter; a launch that gave up may have left them set, so the next call starts clean.
+    cudaMemset(h->d_status, 0, 256);
     if (status & kStatusTimeout) return fail(h, HYAT_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");
     return fail(h, HYAT_ERR_DEVICE_TIMEOUT, "a device-side bounds check failed");
   }

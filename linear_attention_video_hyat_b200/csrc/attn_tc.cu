@@ -57,6 +57,7 @@ constexpr int kRegsLoadMma = 104;
 // The reference max m of a row moves only when the running sum l would leave the safe fp32
 // range: every exponent uses the same m as its row's accumulators, so the result is exact.
 constexpr float kSafeSum = 1.2676506e30f;        // 2^100
+constexpr float kTinySum = 7.8886091e-31f;        // 2^-100
 
 // instruction descriptor, kind::f16: D f32, A/B bf16, M = 128, N = 128
 constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -275,9 +276,12 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
       }
       // Optimistic pass: p = 2^(s * scale_log2 - m) with the row's current reference m.
       float rs = exp_tile(r, sl, -m, tS);
-      // Rare slow path: the sum left the safe range (a score far above m). Move m to the row
-      // max, rescale O and l (after the previous P.V has landed), and redo the tile.
-      if (__any_sync(0xffffffffu, !(l + rs < kSafeSum))) {
+      // Rare slow path: the sum left the safe range. A score far above m: move m up to the
+      // row max. A sum far below 1 (no linear term, every score so far far below m, so the
+      // exponentials approach the flush-to-zero range): move m down to the larger of the row
+      // max and log2 of the sum so far. Then rescale O and l (after the previous P.V has
+      // landed) and redo the tile.
+      if (__any_sync(0xffffffffu, !(l + rs < kSafeSum && l + rs >= kTinySum))) {
         float mx[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -287,8 +291,11 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
           mx[k] = fmaxf(a, u2f(r[k + 120]));
         }
         const float mrow = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], fmax3(mx[5], mx[6], mx[7])));
-        const float m_new = fmaxf(m, mrow * sl);
-        const float alpha = ex2(m - m_new);
+        const bool under = !(l + rs >= kTinySum);
+        const float m_new = under ? fmaxf(mrow * sl, l > 0.0f ? m + __log2f(l) : -INFINITY) : fmaxf(m, mrow * sl);
+        // l = 0: nothing has been added yet, so O holds no weight (a zero linear term, or the
+        // split slot's accumulator before its first P.V, which starts it afresh)
+        const float alpha = l > 0.0f ? ex2(m - m_new) : 0.0f;
         // Rescale O once its last product so far (commit j - 1 + lin of this pair) has
         // landed. On slot 1 of a split pair at j = 0 nothing has been committed yet: the wait
         // is for the previous pair's last phase (already complete), and the values scaled
@@ -662,13 +669,9 @@ static cudaError_t launch_attn_tc_impl(const AttnArgs& a, int32_t* n_pairs_dev, 
   if (!make_map(&mq, a.q, a.q_rows, a.BH) || !make_map(&mk, a.k, a.k_rows, a.BH) ||
       !make_map(&mv, a.v, a.k_rows, a.BH) || !make_map(&ms, a.srest_bf16, D, int64_t(a.BH) * a.nqg))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_set[tc::kMaxDevices];
+  cudaError_t attr_e = tc::set_smem_attr_once(reinterpret_cast<const void*>(attn_tc_kernel), kSmemBytes, attr_set);
+  if (attr_e != cudaSuccess) return attr_e;
   TcParams p{};
   p.work = a.work;
   p.entries = a.entries;

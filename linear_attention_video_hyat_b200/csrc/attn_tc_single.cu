@@ -11,7 +11,7 @@
 //     j mod 2), each with its own partial row sum; the epilogue adds the two sums and each
 //     warpgroup normalises and stores 64 columns of O;
 //   * exponents use the fixed reference m = 0 (p = 2^(s * scale * log2 e)). A query tile
-//     whose row sum leaves the safe fp32 range (>= 2^100, inf or NaN) is appended to a redo
+//     whose row sum leaves the safe fp32 range (>= 2^100 or < 2^-100, inf, NaN) is appended to a redo
 //     list, and attn_tc_kernel, which moves its reference max exactly, recomputes it after
 //     this kernel. For unit-scale inputs the list stays empty;
 //   * phi(Q) (the A operand of the linear-term MMA) sits in S2's first 64 columns until the
@@ -40,6 +40,7 @@ constexpr int NT1 = 384;                         // 3 warpgroups
 constexpr int kRegsSm1 = 184;
 constexpr int kRegsLm1 = 136;
 constexpr float kSafe1 = 1.2676506e30f;          // 2^100
+constexpr float kTiny1 = 7.8886091e-31f;          // 2^-100
 
 // instruction descriptor, kind::f16: D f32, A/B bf16, M = 128, N = 128
 constexpr uint32_t kIdesc1 = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -221,7 +222,10 @@ __device__ __forceinline__ void softmax_single(Smem1* sm, const SingleParams& p,
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int rr = lane + 32 * k;
-        bad |= rr < wi.q_len && !(sm->lsum[0][rr] + sm->lsum[1][rr] < kSafe1);
+        const float sum = sm->lsum[0][rr] + sm->lsum[1][rr];
+        // too large (overflow ahead), or too small: with no linear term a row whose logits
+        // all lie far below 0 flushes its exponentials to zero
+        bad |= rr < wi.q_len && !(sum < kSafe1 && sum >= kTiny1);
       }
       if (__any_sync(0xffffffffu, bad) && lane == 0) {
         const int k = atomicAdd(p.redo_count, 1);
@@ -470,13 +474,9 @@ cudaError_t launch_attn_single(const AttnArgs& a, int32_t* redo_count, int4* red
   if (!make_map(&mq, a.q, a.q_rows, a.BH) || !make_map(&mk, a.k, a.k_rows, a.BH) ||
       !make_map(&mv, a.v, a.k_rows, a.BH) || !make_map(&ms, a.srest_bf16, D, int64_t(a.BH) * a.nqg))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmem1Bytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_set[tc::kMaxDevices];
+  cudaError_t attr_e = tc::set_smem_attr_once(reinterpret_cast<const void*>(attn_single_kernel), kSmem1Bytes, attr_set);
+  if (attr_e != cudaSuccess) return attr_e;
   SingleParams p{};
   p.work = a.work;
   p.entries = a.entries;

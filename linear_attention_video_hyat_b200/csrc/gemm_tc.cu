@@ -234,13 +234,9 @@ cudaError_t launch_complement_tc(const ComplementTcArgs& a, int num_sms, cudaStr
   if (!make_map_cols(&ma, a.cm_bf16, a.nseg_pad, a.nqg, a.mask_heads) ||
       !make_map_cols(&mhi, a.seg_hi, a.E, a.nseg, a.BH) || !make_map_cols(&mlo, a.seg_lo, a.E, a.nseg, a.BH))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_complement_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kGemmSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_set[tc::kMaxDevices];
+  cudaError_t attr_e = tc::set_smem_attr_once(reinterpret_cast<const void*>(gemm_complement_kernel), kGemmSmemBytes, attr_set);
+  if (attr_e != cudaSuccess) return attr_e;
   GemmParams p{};
   p.BH = a.BH;
   p.H = a.H;

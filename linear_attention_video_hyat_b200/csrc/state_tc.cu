@@ -359,13 +359,9 @@ cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t
   static_assert(4 * 64 * TOK * 2 == STAGE_BYTES, "stage bytes must match the four TMA boxes");
   if (!tc::make_map(&mk, a.k, a.rows_per_bh, a.BH, TOK) || !tc::make_map(&mv, a.v, a.rows_per_bh, a.BH, TOK))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(state_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kStateSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<bool> attr_set[tc::kMaxDevices];
+  cudaError_t attr_e = tc::set_smem_attr_once(reinterpret_cast<const void*>(state_tc_kernel), kStateSmemBytes, attr_set);
+  if (attr_e != cudaSuccess) return attr_e;
   const int parts = a.parts > 1 ? a.parts : 1;
   if (parts > 1 && (a.partial == nullptr || a.out_hi != nullptr || a.part_len <= 0)) return cudaErrorInvalidValue;
   StateParams p{};

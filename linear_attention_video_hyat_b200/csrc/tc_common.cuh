@@ -7,6 +7,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <utility>
 
@@ -216,6 +217,22 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// ------------------------------------------------------------------ host: kernel attributes
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) holds per device, so a kernel remembers
+// it per device (the current one). Two threads that race here both set the same value,
+// which is harmless; the flag only saves the call afterwards.
+constexpr int kMaxDevices = 64;
+inline cudaError_t set_smem_attr_once(const void* kernel, size_t bytes, std::atomic<bool> (&done)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess && cached) done[dev].store(true, std::memory_order_release);
+  return e;
 }
 
 // ------------------------------------------------------------------ host: tensor maps

@@ -22,3 +22,18 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "tiny_bidir_f32_T4x64" and "fit in L2" in d["config"]["l2"]
+    assert "cpu_model" in d["cpu_baseline"] and "blas" in d["cpu_baseline"]
+
+
+def test_reference_arm_never_loads_the_library():
+    """The oracle arm counts its FLOPs from the oracle's own rules and must not map libhyat.so."""
+    code = ("import sys; sys.argv = ['bench.py', '--impl', 'reference', '--steps', '1', '--warmup', '0', "
+            "'--workload', 'wan1.3b_bidir_T21x1560']; import bench; bench.main(); "
+            "maps = open('/proc/self/maps').read(); "
+            "print('LOADED' if ('libhyat' in maps or 'linear_attention_video_hyat_b200.hyat' in sys.modules) "
+            "else 'CLEAN')")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip().splitlines()[-1] == "CLEAN"
+    d = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][0])
+    assert d["impl"] == "reference" and d["value"] > 0
