@@ -63,8 +63,11 @@ def parse():
                    help="tensor-core attention schedule of the bidirectional modes: a pair of query "
                         "tiles per CTA (default) or one query tile per CTA (HYAT_FLAG_SINGLE_TILE)")
     p.add_argument("--rope", action="store_true",
-                   help="streaming workload: each step first applies the capped temporal RoPE "
-                        "(hyat_rope_temporal) to the chunk's Q and K")
+                   help="streaming workload: the capped temporal RoPE of the chunk's Q and K fused "
+                        "into each step (hyat_config.rope_t_dims)")
+    p.add_argument("--graph", action="store_true",
+                   help="streaming workload: device step masks, steady steps replayed from the "
+                        "library's CUDA graphs (hyat_fwd_stream_step_graph)")
     return p.parse_args()
 
 
@@ -384,62 +387,56 @@ def bench_stream(a, w, rank, world, local):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    cfg = hyat.config_from_workload(w, mask_heads=w.H)
-    dev_in = [(q.to(dev), k.to(dev), v.to(dev), m) for q, k, v, m in inputs]
+    cfg = hyat.config_from_workload(w, mask_heads=w.H, rope=ROPE if a.rope else None)
+    if a.graph:
+        config["graph"] = "device masks; steady steps replayed from the library's CUDA graphs"
+    dev_in = [(q.to(dev), k.to(dev), v.to(dev), m, torch.from_numpy(np.ascontiguousarray(m)).to(dev))
+              for q, k, v, m in inputs]
     od = torch.empty_like(dev_in[0][0])
     stream = torch.cuda.current_stream(dev)
 
-    n_sink = w.sink_frames // w.chunk_frames
-    qr, kr = torch.empty_like(od), torch.empty_like(od)
-    rope_events = []
+    def step(h, x, m_host, s_, out):
+        q, k, v, m, md = x
+        if s_ < nwc:          # the window is still filling: masks of the growing shape
+            m = wl.gen_stream_step(w, s_, seed=w.seed + rank)[3]
+            md = torch.from_numpy(np.ascontiguousarray(m)).to(dev)
+        if a.graph:
+            h.stream_step_dev(q, k, v, mask=md, out=out, graph=True)
+        else:
+            h.stream_step(q, k, v, mask=m if m_host is None else m_host, out=out)
 
-    def rope(q, k, s, timed=False):
-        """The step before attention: Q and K of chunk s turned by their capped offsets from
-        the oldest window chunk's first frame."""
-        f0 = s * w.chunk_frames
-        ref = max(n_sink, s - nwc + 1) * w.chunk_frames
-        if timed:
-            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            ev[0].record(stream)
-        for x, y in ((q, qr), (k, kr)):
-            hyat.rope_temporal(x, w.tokens_per_frame, f0, ref, ROPE["cap"], ROPE["t_dims"], ROPE["base"], out=y)
-        if timed:
-            ev[1].record(stream)
-            rope_events.append(ev)
-        return qr, kr
-
-    def run(h, steps, first, timed=False):
+    def run(h, steps, first):
         for i in range(steps):
-            s = first + i
-            q, k, v, m = dev_in[s % n_dist]
-            if s < nwc:       # the window is still filling: masks of the growing shape
-                m = wl.gen_stream_step(w, s, seed=w.seed + rank)[3]
-            if a.rope:
-                q, k = rope(q, k, s, timed)
-            h.stream_step(q, k, v, mask=m, out=od)
+            s_ = first + i
+            step(h, dev_in[s_ % n_dist], None, s_, od)
 
     h = hyat.Hyat(cfg, device=dev)
-    run(h, warm, 0)
+    run(h, warm + n_dist * nwc, 0)        # warm-up (and, with --graph, one capture per phase and input set)
     h.sync()
+    first = warm + n_dist * nwc
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    host0 = time.perf_counter()
     with ClockSampler(local) as clk:
         t0.record(stream)
-        run(h, a.steps, warm)
+        run(h, a.steps, first)
         t1.record(stream)
+        host_s = time.perf_counter() - host0
         torch.cuda.synchronize(dev)
     h.sync()
     ms = max_over_ranks(t0.elapsed_time(t1) / a.steps, dev)
-    h.set_profiling(True)
+    first += a.steps
+    h.set_profiling(True)        # per-launch events (graph replay is off while profiling)
     h.kernel_times()
     with ClockSampler(local) as clk2:
-        run(h, a.steps, warm + a.steps, timed=True)
+        run(h, a.steps, first)
         torch.cuda.synchronize(dev)
+    first += a.steps
     kt = h.kernel_times()
     h.set_profiling(False)
-    launches = sum(n for _, n in kt.values()) + 2 * len(rope_events)
+    launches = sum(n for _, n in kt.values())
     value, tokens_per_s = job_throughput(mean_flops, w.B * w.chunk_tokens, ms, world)
     pk, pk_src = peaks()
     attn_ms = kt["attention"][0] / max(kt["attention"][1], 1)
@@ -452,42 +449,79 @@ def bench_stream(a, w, rank, world, local):
                 "frac_sustained": achieved / pk["bf16_tflops_sustained"], "traffic": None,
                 "launch_ms": attn_ms, "algorithmic_flops_per_launch": mean_attn}
     kernels = {k_: {"ms_per_launch": t_ / max(n_, 1), "launches": n_} for k_, (t_, n_) in kt.items() if n_}
-    if rope_events:
-        r_ms = sum(e0.elapsed_time(e1) for e0, e1 in rope_events) / (2 * len(rope_events))
-        r_bytes = 2 * od.numel() * od.element_size()        # out of place: one read, one write
-        kernels["rope"] = {"ms_per_launch": r_ms, "launches": 2 * len(rope_events),
-                           "hbm_gbs": r_bytes / (r_ms / 1e3) / 1e9,
-                           "timing": "CUDA events around the Q and K calls of each step, pass 2"}
+    if "prep" in kernels:
+        # the prep kernel moves the chunk's K and V into the ring (read + write) and, with the
+        # fused RoPE, Q into its turned copy; plus the fold's partial states it sums
+        E = w.d * w.d + w.d
+        kv = w.B * w.H * w.chunk_tokens * w.d * 2
+        pbytes = 4 * kv + (2 * kv if a.rope else 0)
+        kernels["prep"]["algorithmic_bytes"] = pbytes
+        kernels["prep"]["hbm_gbs"] = pbytes / (kernels["prep"]["ms_per_launch"] / 1e3) / 1e9
+    config["host_ms_per_step"] = 1e3 * host_s / a.steps
 
     e2e = None
     if not a.no_e2e:
-        pinned = [tuple(t.pin_memory() for t in x[:3]) + (x[3],) for x in inputs]
-        oh = torch.empty_like(pinned[0][0]).pin_memory()
-        qd, kd, vd = (torch.empty_like(t) for t in dev_in[0][:3])
-        e_steps = max(3, min(a.steps, 20))
+        # H2D of the step's Q, K, V (pinned) and its mask, the step, D2H of its output; steps
+        # run in order on the compute stream (each needs the ring the previous one wrote), while
+        # step i+1's inputs and step i-1's output cross PCIe (double-buffered device tensors,
+        # one copy stream per direction)
+        pinned = [tuple(t.pin_memory() for t in x[:3]) for x in inputs]
+        host_masks = [torch.from_numpy(np.ascontiguousarray(x[3])).pin_memory() for x in inputs]
+        host_out = [torch.empty_like(pinned[0][0]).pin_memory() for _ in range(2)]
+        dbuf = [tuple(torch.empty_like(t) for t in dev_in[0][:3]) for _ in range(2)]
+        dmask = [torch.empty_like(dev_in[0][4]) for _ in range(2)]
+        dout = [od, torch.empty_like(od)]
+        e_steps = max(4, min(a.steps, 20))
+        counter = [first]
 
-        def run_e2e(first, steps):
+        def e2e_run(steps):
+            h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+            ev = lambda: torch.cuda.Event()
+            in_free, in_ready, out_ready, out_free = ([ev(), ev()] for _ in range(4))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            h2d.wait_event(e0)
+            d2h.wait_event(e0)
             for i in range(steps):
-                qh, kh_, vh, m = pinned[(first + i) % n_dist]
-                qd.copy_(qh, non_blocking=True); kd.copy_(kh_, non_blocking=True); vd.copy_(vh, non_blocking=True)
-                qx, kx = rope(qd, kd, warm + 2 * a.steps + first + i) if a.rope else (qd, kd)
-                h.stream_step(qx, kx, vd, mask=m, out=od)
-                oh.copy_(od, non_blocking=True)
-        run_e2e(0, 2)
-        torch.cuda.synchronize(dev)
+                b, j = i % 2, counter[0] % n_dist
+                with torch.cuda.stream(h2d):
+                    if i >= 2:
+                        h2d.wait_event(in_free[b])
+                    for dst, src in zip(dbuf[b], pinned[j]):
+                        dst.copy_(src, non_blocking=True)
+                    dmask[b].copy_(host_masks[j], non_blocking=True)
+                    in_ready[b].record(h2d)
+                stream.wait_event(in_ready[b])
+                if i >= 2:
+                    stream.wait_event(out_free[b])
+                q, k, v = dbuf[b]
+                if a.graph:
+                    h.stream_step_dev(q, k, v, mask=dmask[b], out=dout[b], graph=True)
+                else:
+                    h.stream_step_dev(q, k, v, mask=dmask[b], out=dout[b])
+                counter[0] += 1
+                in_free[b].record(stream)
+                out_ready[b].record(stream)
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(out_ready[b])
+                    host_out[b].copy_(dout[b], non_blocking=True)
+                    out_free[b].record(d2h)
+            for b in range(2):
+                stream.wait_event(out_free[b])
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            return e0.elapsed_time(e1) / steps
+        e2e_run(2 * nwc * 2)                        # warm-up (captures for the double buffers)
         if world > 1:
             torch.distributed.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        run_e2e(2, e_steps)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ems = max_over_ranks(e0.elapsed_time(e1) / e_steps, dev)
+        ems = max_over_ranks(e2e_run(e_steps), dev)
         e_value, e_tokens = job_throughput(mean_flops, w.B * w.chunk_tokens, ems, world)
         q0 = inputs[0][0]
         e2e = {"value": e_value, "unit": "TFLOP/s", "ms_per_step": ems, "tokens_per_s": e_tokens,
                "h2d_bytes_per_step": 3 * q0.numel() * q0.element_size() + int(inputs[0][3].nbytes),
-               "d2h_bytes_per_step": q0.numel() * q0.element_size()}
+               "d2h_bytes_per_step": q0.numel() * q0.element_size(),
+               "overlap": "steps in order; the next step's H2D and the previous step's D2H overlap "
+                          "the step (double-buffered device tensors, one copy stream per direction)"}
     if world > 1:
         torch.distributed.barrier()
     if rank == 0:

@@ -118,6 +118,18 @@ typedef struct {
   float scale;                   /* softmax logit scale; 0 => 1/sqrt(d) */
   int32_t sink_frames;           /* STREAM: leading frames kept in the window for good (an
                                     attention sink); a multiple of chunk_frames, 0 = none */
+  /* STREAM: the capped temporal RoPE of hyat_rope_temporal, fused into the step (Long-Horizon
+   * Streaming Video Generation via Hybrid Attention with Decoupled Distillation, Section 2.C,
+   * the relative RoPE constraint). rope_t_dims = 0: none. Otherwise each call turns the first
+   * rope_t_dims dimensions of its Q and K exactly as hyat_rope_temporal would, with the
+   * reference frame the first frame of the oldest rolling-window chunk (the call's own chunk
+   * while the window holds none yet) and the index capped at rope_cap - 1: K on its way into
+   * the KV ring, Q into a workspace copy that the attention reads. The caller's Q and K are
+   * not modified. Needs rope_t_dims even and <= d, rope_cap >= 1, chunk_frames * rope_t_dims
+   * <= 8192. */
+  int32_t rope_t_dims;
+  int32_t rope_cap;
+  float rope_base;               /* frequency base; 0 => 10000 */
 } hyat_config;
 
 typedef struct hyat_ctx* hyat_handle;
@@ -164,6 +176,25 @@ HYAT_API hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const vo
 HYAT_API hyat_status hyat_fwd_stream_denoise(hyat_handle h, const void* q, const void* k, const void* v,
                                     void* o, const uint8_t* host_step_mask, void* stream);
 
+/* hyat_fwd_stream_step with the step mask already in device memory: `dev_step_mask` has the
+ * layout of host_step_mask (NULL = every tile kept) and must stay valid until the step has
+ * run. Nothing is copied from the host, so the call can be captured in a CUDA graph by the
+ * library (hyat_fwd_stream_step_graph). The diagonal tiles are checked on the device: a
+ * missing one is computed as given and reported by hyat_sync() as HYAT_ERR_INVALID_ARG. */
+HYAT_API hyat_status hyat_fwd_stream_step_dev(hyat_handle h, const void* q, const void* k, const void* v,
+                                     void* o, const uint8_t* dev_step_mask, void* stream);
+
+/* hyat_fwd_stream_step_dev replayed from a CUDA graph. Once the window is full, a step's
+ * launches depend only on its ring phase (step mod window_frames / chunk_frames) and on the
+ * pointers q, k, v, o and dev_step_mask: the first such step of each phase is captured (on a
+ * stream of the handle) into a graph, and later steps of that phase with the same pointers
+ * launch the graph on `stream` with one call. New pointers capture again; the handle keeps
+ * the 16 most recent graphs, so a caller that rotates a few input buffers reuses them. Steps
+ * before the window is full, and calls with profiling on, run as hyat_fwd_stream_step_dev.
+ * Results equal hyat_fwd_stream_step_dev's bit for bit. */
+HYAT_API hyat_status hyat_fwd_stream_step_graph(hyat_handle h, const void* q, const void* k, const void* v,
+                                       void* o, const uint8_t* dev_step_mask, void* stream);
+
 /* Wait for the last call's stream and report device-side errors. */
 HYAT_API hyat_status hyat_sync(hyat_handle h);
 
@@ -209,6 +240,16 @@ HYAT_API hyat_status hyat_lvsa_mask(int32_t n_frames, int32_t tokens_per_frame, 
 HYAT_API hyat_status hyat_stream_plan(const hyat_config* cfg, int32_t step, int32_t* info,
                              size_t info_len);
 
+/* Test hook (STREAM): the layout the last streaming call built on the device, copied to the
+ * host (synchronises the device). work: n_work x 8 int32 per (b, h, query tile)
+ * {bh, q_row, q_len, 0, entry_begin, entry_end, 0, 0}; entries: n_work x cap slots of 2 int32
+ * {k_row, k_len}, item t's key tiles at [entry_begin, entry_end), k_row a row of the KV ring
+ * (slot * L + offset in the chunk); info (4 + ring slots int32): hyat_stream_plan of that
+ * call's step. counts[0] = n_work, counts[1] = entry slots, counts[2] = that step. Null
+ * arrays: counts only. HYAT_ERR_STATE before the first streaming call. */
+HYAT_API hyat_status hyat_stream_get_layout(hyat_handle h, int32_t* work, size_t work_cap, int32_t* entries,
+                                   size_t entries_cap, int32_t* info, size_t info_len, int64_t* counts);
+
 /* Stream state (S, z, KV ring, step, and whether the current chunk's fold
  * has run) to / from a host buffer: a 48-byte header, then S, z as fp32
  * [B*H][d*d + d], then the K and V rings. The size is
@@ -220,7 +261,8 @@ HYAT_API hyat_status hyat_stream_set_state(hyat_handle h, const void* src_host, 
 /* Kernel timing: when enabled, each forward call records CUDA events around
  * its launches; hyat_kernel_times() returns the summed milliseconds and
  * launch counts per kernel kind since the last reset (kinds: 0 state,
- * 1 complement, 2 attention, 3 stream fold + ring copy, 4 layout/prep).
+ * 1 complement, 2 attention, 3 stream fold, 4 stream prep: fold reduce, ring copy, fused
+ * RoPE and layout).
  * Reading the times synchronises the device. */
 HYAT_API hyat_status hyat_set_profiling(hyat_handle h, int enable);
 HYAT_API hyat_status hyat_kernel_times(hyat_handle h, double* ms, int64_t* launches, int n_kinds);
@@ -235,13 +277,17 @@ HYAT_API hyat_status hyat_kernel_times(hyat_handle h, double* ms, int64_t* launc
  * Same operation and tensor conventions as hyat_fwd_bidir, for WINDOW and
  * RADIAL configurations, without a handle or a workspace: the scratch lives in
  * one static 32 MiB __device__ array that every GPU loading the library holds
- * until the process exits. No cudaMalloc, cudaFree or allocating library call
- * is made. Returns HYAT_ERR_UNSUPPORTED when the configuration needs more than
+ * until the process exits. It runs the same kernels, in the same order and with
+ * the same work order, as hyat_fwd_bidir on a handle of the same configuration,
+ * so its output equals that call's bit for bit. No cudaMalloc, cudaFree or
+ * allocating library call is made. Returns HYAT_ERR_UNSUPPORTED when the configuration needs more than
  * 32 MiB of scratch (for example, 12 heads x 21 frames of 1560 tokens at
  * d = 128 need about 25 MiB), HYAT_ERR_INVALID_ARG for other modes, bad
  * configurations or pointers that are not 16-byte aligned.
  * The first call on a device resolves the array's device address; make that
- * first call before any stream capture. Every call reuses the same array and
+ * first call before any stream capture. The call copies its layout tables from
+ * host memory that it releases on return, so it returns HYAT_ERR_UNSUPPORTED
+ * (nothing enqueued) when `stream` is being captured. Every call reuses the same array and
  * leaves the previous call's contents in it (the status word is cleared on
  * each call): calls that overlap on the GPU -- on different streams, or from
  * different threads -- race on it and must be serialised by the caller.

@@ -15,7 +15,7 @@ using namespace hyat;
 
 namespace {
 
-constexpr int kKinds = 5;  // state, complement, attention, fold+ring, layout/prep
+constexpr int kKinds = 5;  // state, complement, attention, stream fold, stream prep
 enum Kind { K_STATE = 0, K_COMPLEMENT = 1, K_ATTN = 2, K_FOLD = 3, K_PREP = 4 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -23,7 +23,7 @@ int32_t nseg_pad64(int32_t n) { return (n + 63) / 64 * 64; }
 
 struct Plan {
   size_t status = 0, work = 0, entries = 0, pairs = 0, cm = 0, cm_bf16 = 0, sseg = 0, srest = 0, srest_bf16 = 0;
-  size_t ring_k = 0, ring_v = 0, mask = 0, fold_partial = 0, redo = 0, total = 0;
+  size_t ring_k = 0, ring_v = 0, mask = 0, fold_partial = 0, q_rot = 0, redo = 0, total = 0;
   int64_t n_work = 0, n_entries = 0;
 };
 
@@ -61,6 +61,7 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
     p.ring_v = take(size_t(BH * slots * Lc * c.d * elem_bytes(c)));
     p.mask = take(size_t(c.mask_heads) * nqt * nqt * slots);
     p.fold_partial = take(sizeof(float) * BH * fold_parts_cap(c) * E);
+    if (c.rope_t_dims > 0) p.q_rot = take(size_t(BH * Lc * c.d * elem_bytes(c)));
   } else {
     p.cm = take(sizeof(float) * size_t(L.cm_heads) * L.nqg * L.nseg);
     if (c.mode == HYAT_MODE_BLOCKMASK || c.mode == HYAT_MODE_RADIAL)
@@ -131,6 +132,18 @@ struct hyat_ctx {
   uint8_t* d_mask = nullptr;
   int32_t step = 0;
   int32_t folded_step = -1;          // step whose evicted chunk is already in S, z
+  int32_t last_step = -1;            // step of the last streaming call (its layout is on the device)
+  void* d_q_rot = nullptr;           // fused RoPE: the turned Q of the current call
+  double rope_theta[64] = {};        // fused RoPE: base^(-2i / t_dims)
+  // graph replay of steady streaming steps: one captured step per (ring phase, fold, pointers)
+  struct StepGraph {
+    cudaGraphExec_t exec;
+    int32_t phase;
+    bool fold;
+    const void *q, *k, *v, *o, *mask;
+  };
+  std::vector<StepGraph> graphs;
+  cudaStream_t cap_stream = nullptr;
   float* d_fold_partial = nullptr;
   int32_t fold_parts = 1, fold_part_len = 0;
   bool use_tc = false;
@@ -294,6 +307,11 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
     h->d_ring_v = ws + h->plan.ring_v;
     h->d_mask = reinterpret_cast<uint8_t*>(ws + h->plan.mask);
     h->d_fold_partial = reinterpret_cast<float*>(ws + h->plan.fold_partial);
+    if (h->plan.q_rot) h->d_q_rot = ws + h->plan.q_rot;
+    if (cfg->rope_t_dims > 0) {
+      const double base = cfg->rope_base > 0.0f ? static_cast<double>(cfg->rope_base) : 10000.0;
+      for (int i = 0; i < cfg->rope_t_dims / 2; ++i) h->rope_theta[i] = std::pow(base, -2.0 * i / cfg->rope_t_dims);
+    }
   } else {
     h->d_cm = reinterpret_cast<float*>(ws + h->plan.cm);
     if (h->plan.cm_bf16) h->d_cm_bf16 = reinterpret_cast<uint16_t*>(ws + h->plan.cm_bf16);
@@ -375,6 +393,8 @@ hyat_status hyat_destroy(hyat_handle h) {
     cudaEventDestroy(r.b);
   }
   for (auto e : h->free_events) cudaEventDestroy(e);
+  for (auto& g : h->graphs) cudaGraphExecDestroy(g.exec);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   delete h;
   return HYAT_OK;
 }
@@ -427,12 +447,65 @@ hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const vo
 
 namespace {
 
+// Launches of one streaming call for the current chunk, all on `s` and all capturable: the
+// fold of the chunk leaving the window (if `fold`), the prep kernel (fold reduce, K and V into
+// the ring slot, the fused RoPE, the step's layout from the device mask `mask`), then the
+// attention. Every argument is a function of the step's ring phase once the window is full.
+hyat_status enqueue_stream_call(hyat_handle h, const void* q, const void* k, const void* v, void* o,
+                                const uint8_t* mask, bool fold, const StreamGeometry& g, int32_t step,
+                                cudaStream_t s) {
+  const hyat_config& c = h->cfg;
+  const int32_t Lc = stream_chunk_tokens(c), nwc = stream_window_chunks(c), nqt = tiles(Lc);
+  const int32_t slot = g.write_slot;
+  cudaError_t e = timed(h, K_FOLD, s, [&]() -> cudaError_t {
+    if (!fold) return cudaSuccess;
+    // chunk s - nwc leaves the window: its slot is the one this call writes
+    SegStateArgs sa{};
+    sa.k = h->d_ring_k; sa.v = h->d_ring_v; sa.rows_per_bh = h->rk;
+    sa.BH = h->BH; sa.d = c.d; sa.dtype = c.dtype; sa.phi = c.phi;
+    sa.nseg = 1; sa.seg_base = slot * Lc; sa.seg_stride = Lc; sa.seg_len = Lc;
+    sa.out = h->d_srest; sa.accumulate = 1; sa.status = h->d_status;
+    if (!h->use_tc) return launch_seg_state(sa, s);
+    // token ranges in parallel; the prep kernel sums them in order into S, z
+    sa.parts = h->fold_parts; sa.part_len = h->fold_part_len; sa.partial = h->d_fold_partial;
+    return launch_seg_state_tc(sa, h->num_sms, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(h, e, "stream fold");
+  StreamPrepArgs pa{};
+  pa.BH = h->BH; pa.L = Lc; pa.d = c.d; pa.elem_bytes = static_cast<int32_t>(elem_bytes(c));
+  if (fold && h->use_tc) {
+    pa.partial = h->d_fold_partial; pa.srest = h->d_srest; pa.srest_bf16 = h->d_srest_bf16; pa.parts = h->fold_parts;
+  }
+  pa.k = k; pa.v = v; pa.ring_k = h->d_ring_k; pa.ring_v = h->d_ring_v;
+  pa.nslots = stream_ring_slots(c); pa.slot = slot;
+  if (c.rope_t_dims > 0) {
+    pa.q = q; pa.q_out = h->d_q_rot;
+    pa.half_t = c.rope_t_dims / 2; pa.chunk_frames = c.chunk_frames; pa.tokens_per_frame = c.tokens_per_frame;
+    // offset of the chunk's first frame from the first frame of the oldest rolling-window
+    // chunk (0 while the window holds none yet: a sink chunk at its own step)
+    pa.p0 = step >= g.first_window ? (step - g.first_window) * c.chunk_frames : 0;
+    pa.cap = c.rope_cap;
+    for (int i = 0; i < pa.half_t; ++i) pa.theta[i] = h->rope_theta[i];
+  }
+  pa.mask = mask; pa.work = h->d_work; pa.entries = h->d_entries; pa.status = h->d_status;
+  pa.H = c.H; pa.mask_heads = c.mask_heads; pa.nqt = nqt; pa.nkt = nqt * g.n_visible;
+  pa.cap_entries = nqt * stream_ring_slots(c); pa.nwc = nwc;
+  pa.n_sink_visible = g.n_sink_visible; pa.first_window_mod = g.first_window % nwc;
+  e = timed(h, K_PREP, s, [&] { return launch_stream_prep(pa, h->num_sms, s); });
+  if (e != cudaSuccess) return cuda_fail(h, e, "stream prep kernel");
+  const void* qa = c.rope_t_dims > 0 ? h->d_q_rot : q;
+  return launch_attention(h, attn_args(h, qa, h->d_ring_k, h->d_ring_v, o, int64_t(h->BH) * nqt, 1), s);
+}
+
+enum class MaskSrc { kHost, kDevice, kGraph };
+constexpr size_t kMaxStepGraphs = 16;
+
 // One streaming call for the current chunk. The first call of a chunk folds the chunk that
 // leaves the window into S, z; every call writes its K, V into the chunk's ring slot and
 // attends. `commit` marks the chunk's final call: the step counter then advances, and the
 // K, V just written stay in the window.
 hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void* v, void* o,
-                        const uint8_t* host_step_mask, void* stream, bool commit) {
+                        const uint8_t* step_mask, MaskSrc src, void* stream, bool commit) {
   if (!h) return HYAT_ERR_INVALID_ARG;
   if (h->cfg.mode != HYAT_MODE_STREAM) return fail(h, HYAT_ERR_INVALID_ARG, "handle is not in STREAM mode");
   hyat_status st = check_ptrs(h, q, k, v, o);
@@ -441,64 +514,69 @@ hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void*
   const int32_t Lc = stream_chunk_tokens(c), nwc = stream_window_chunks(c), nqt = tiles(Lc);
   const int32_t s_ = h->step;
   const StreamGeometry g = stream_geometry(c, s_);
-  const int32_t nwin = g.n_visible;
-  const int32_t nkt = nqt * nwin;
+  const int32_t nkt = nqt * g.n_visible;
   const size_t mask_bytes = size_t(c.mask_heads) * nqt * nkt;
-  if (host_step_mask) {
+  if (src == MaskSrc::kHost && step_mask) {
     for (int32_t m = 0; m < c.mask_heads; ++m)
       for (int32_t i = 0; i < nqt; ++i)
-        if (!host_step_mask[(size_t(m) * nqt + i) * nkt + nqt * (nwin - 1) + i])
+        if (!step_mask[(size_t(m) * nqt + i) * nkt + nqt * (g.n_visible - 1) + i])
           return fail(h, HYAT_ERR_INVALID_ARG, "step mask: diagonal tile of the newest chunk must be kept");
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   h->last_stream = s;
-  cudaError_t e;
-  if (host_step_mask)
-    e = cudaMemcpyAsync(h->d_mask, host_step_mask, mask_bytes, cudaMemcpyHostToDevice, s);
-  else
-    e = cudaMemsetAsync(h->d_mask, 1, mask_bytes, s);
-  if (e != cudaSuccess) return cuda_fail(h, e, "step mask upload");
-  const int32_t slot = g.write_slot;
   const bool fold = g.evicted >= 0 && h->folded_step != s_;
-  e = timed(h, K_FOLD, s, [&]() -> cudaError_t {
-    if (fold) {  // chunk s - nwc leaves the window: fold it into S, z (its slot is the one now written)
-      SegStateArgs sa{};
-      sa.k = h->d_ring_k; sa.v = h->d_ring_v; sa.rows_per_bh = h->rk;
-      sa.BH = h->BH; sa.d = c.d; sa.dtype = c.dtype; sa.phi = c.phi;
-      sa.nseg = 1; sa.seg_base = slot * Lc; sa.seg_stride = Lc; sa.seg_len = Lc;
-      sa.out = h->d_srest; sa.accumulate = 1; sa.status = h->d_status;
-      if (h->use_tc) {
-        // token ranges in parallel, then an ordered sum into S, z and the bf16 copy
-        sa.parts = h->fold_parts; sa.part_len = h->fold_part_len; sa.partial = h->d_fold_partial;
-        cudaError_t e2 = launch_seg_state_tc(sa, h->num_sms, s);
-        if (e2 != cudaSuccess) return e2;
-        FoldReduceArgs fa{};
-        fa.partial = h->d_fold_partial; fa.srest = h->d_srest; fa.srest_bf16 = h->d_srest_bf16;
-        fa.BH = h->BH; fa.parts = h->fold_parts; fa.d = c.d;
-        e2 = launch_fold_reduce(fa, s);
-        if (e2 != cudaSuccess) return e2;
-      } else {
-        cudaError_t e2 = launch_seg_state(sa, s);
-        if (e2 != cudaSuccess) return e2;
+  const bool steady = g.n_window == nwc && g.n_sink_visible == stream_sink_chunks(c);
+  if (src == MaskSrc::kGraph && steady && !h->profiling) {
+    const int32_t phase = s_ % nwc;
+    auto it = std::find_if(h->graphs.begin(), h->graphs.end(), [&](const hyat_ctx::StepGraph& x) {
+      return x.phase == phase && x.fold == fold && x.q == q && x.k == k && x.v == v && x.o == o && x.mask == step_mask;
+    });
+    if (it == h->graphs.end()) {
+      // capture this step; the cache keeps the kMaxStepGraphs most recent captures (callers
+      // that rotate a few input buffers reuse one graph per phase and buffer set)
+      if (h->graphs.size() >= kMaxStepGraphs) {
+        cudaGraphExecDestroy(h->graphs.front().exec);
+        h->graphs.erase(h->graphs.begin());
       }
+      cudaError_t e = cudaSuccess;
+      if (!h->cap_stream) e = cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking);
+      if (e != cudaSuccess) return cuda_fail(h, e, "capture stream");
+      e = cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal);
+      if (e != cudaSuccess) return cuda_fail(h, e, "begin capture");
+      if (!step_mask) e = cudaMemsetAsync(h->d_mask, 1, mask_bytes, h->cap_stream);
+      st = e == cudaSuccess
+               ? enqueue_stream_call(h, q, k, v, o, step_mask ? step_mask : h->d_mask, fold, g, s_, h->cap_stream)
+               : cuda_fail(h, e, "step mask fill");
+      cudaGraph_t graph = nullptr;
+      const cudaError_t e2 = cudaStreamEndCapture(h->cap_stream, &graph);
+      if (st != HYAT_OK) {
+        if (graph) cudaGraphDestroy(graph);
+        return st;
+      }
+      if (e2 != cudaSuccess) return cuda_fail(h, e2, "end capture");
+      cudaGraphExec_t exec = nullptr;
+      e = cudaGraphInstantiate(&exec, graph, 0);
+      cudaGraphDestroy(graph);
+      if (e != cudaSuccess) return cuda_fail(h, e, "graph instantiate");
+      h->graphs.push_back({exec, phase, fold, q, k, v, o, step_mask});
+      it = h->graphs.end() - 1;
     }
-    RingCopyArgs ra{};
-    ra.k = k; ra.v = v; ra.ring_k = h->d_ring_k; ra.ring_v = h->d_ring_v;
-    ra.BH = h->BH; ra.L = Lc; ra.d = c.d; ra.nslots = stream_ring_slots(c); ra.slot = slot;
-    ra.elem_bytes = static_cast<int32_t>(elem_bytes(c));
-    return launch_ring_copy(ra, s);
-  });
-  if (e != cudaSuccess) return cuda_fail(h, e, "stream fold / ring copy");
+    const cudaError_t e = cudaGraphLaunch(it->exec, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "graph launch");
+  } else {
+    const uint8_t* m = step_mask;
+    cudaError_t e = cudaSuccess;
+    if (src == MaskSrc::kHost && step_mask)
+      e = cudaMemcpyAsync(h->d_mask, step_mask, mask_bytes, cudaMemcpyHostToDevice, s);
+    else if (!step_mask)
+      e = cudaMemsetAsync(h->d_mask, 1, mask_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "step mask upload");
+    if (src == MaskSrc::kHost || !step_mask) m = h->d_mask;
+    st = enqueue_stream_call(h, q, k, v, o, m, fold, g, s_, s);
+    if (st != HYAT_OK) return st;
+  }
   if (fold) h->folded_step = s_;
-  StreamLayoutArgs la{};
-  la.mask = h->d_mask; la.work = h->d_work; la.entries = h->d_entries;
-  la.BH = h->BH; la.H = c.H; la.mask_heads = c.mask_heads; la.nqt = nqt; la.nkt = nkt;
-  la.cap = nqt * stream_ring_slots(c); la.L = Lc; la.nwc = nwc;
-  la.n_sink_visible = g.n_sink_visible; la.first_window = g.first_window;
-  e = timed(h, K_PREP, s, [&] { return launch_stream_layout(la, s); });
-  if (e != cudaSuccess) return cuda_fail(h, e, "stream layout kernel");
-  st = launch_attention(h, attn_args(h, q, h->d_ring_k, h->d_ring_v, o, int64_t(h->BH) * nqt, 1), s);
-  if (st != HYAT_OK) return st;
+  h->last_step = s_;
   if (commit) h->step += 1;
   return HYAT_OK;
 }
@@ -507,12 +585,44 @@ hyat_status stream_call(hyat_handle h, const void* q, const void* k, const void*
 
 hyat_status hyat_fwd_stream_step(hyat_handle h, const void* q, const void* k, const void* v, void* o,
                                  const uint8_t* host_step_mask, void* stream) {
-  return stream_call(h, q, k, v, o, host_step_mask, stream, true);
+  return stream_call(h, q, k, v, o, host_step_mask, MaskSrc::kHost, stream, true);
 }
 
 hyat_status hyat_fwd_stream_denoise(hyat_handle h, const void* q, const void* k, const void* v, void* o,
                                     const uint8_t* host_step_mask, void* stream) {
-  return stream_call(h, q, k, v, o, host_step_mask, stream, false);
+  return stream_call(h, q, k, v, o, host_step_mask, MaskSrc::kHost, stream, false);
+}
+
+hyat_status hyat_fwd_stream_step_dev(hyat_handle h, const void* q, const void* k, const void* v, void* o,
+                                     const uint8_t* dev_step_mask, void* stream) {
+  return stream_call(h, q, k, v, o, dev_step_mask, MaskSrc::kDevice, stream, true);
+}
+
+hyat_status hyat_fwd_stream_step_graph(hyat_handle h, const void* q, const void* k, const void* v, void* o,
+                                       const uint8_t* dev_step_mask, void* stream) {
+  return stream_call(h, q, k, v, o, dev_step_mask, MaskSrc::kGraph, stream, true);
+}
+
+hyat_status hyat_stream_get_layout(hyat_handle h, int32_t* work, size_t work_cap, int32_t* entries,
+                                   size_t entries_cap, int32_t* info, size_t info_len, int64_t* counts) {
+  if (!h || !counts) return HYAT_ERR_INVALID_ARG;
+  if (h->cfg.mode != HYAT_MODE_STREAM) return fail(h, HYAT_ERR_INVALID_ARG, "handle is not in STREAM mode");
+  if (h->last_step < 0) return fail(h, HYAT_ERR_STATE, "no streaming call yet");
+  const int32_t nqt = tiles(stream_chunk_tokens(h->cfg)), slots = stream_ring_slots(h->cfg);
+  const int64_t n_work = int64_t(h->BH) * nqt, n_ent = n_work * nqt * slots;
+  counts[0] = n_work;
+  counts[1] = n_ent;
+  counts[2] = h->last_step;
+  if (!work || !entries || !info) return HYAT_OK;
+  if (work_cap < size_t(n_work) * 8 || entries_cap < size_t(n_ent) * 2)
+    return fail(h, HYAT_ERR_INVALID_ARG, "layout buffers too small");
+  if (hyat_stream_plan(&h->cfg, h->last_step, info, info_len) != HYAT_OK)
+    return fail(h, HYAT_ERR_INVALID_ARG, "info buffer too small");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(work, h->d_work, sizeof(WorkItem) * n_work, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(entries, h->d_entries, sizeof(Entry) * n_ent, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "layout copy");
+  return HYAT_OK;
 }
 
 hyat_status hyat_sync(hyat_handle h) {
@@ -527,7 +637,8 @@ hyat_status hyat_sync(hyat_handle h) {
     // counter; a launch that gave up may have left them set, so the next call starts clean.
     cudaMemset(h->d_status, 0, 256);
     if (status & kStatusTimeout) return fail(h, HYAT_ERR_DEVICE_TIMEOUT, "a device-side wait timed out");
-    return fail(h, HYAT_ERR_DEVICE_TIMEOUT, "a device-side bounds check failed");
+    if (status & kStatusBadTile) return fail(h, HYAT_ERR_DEVICE_TIMEOUT, "a device-side bounds check failed");
+    return fail(h, HYAT_ERR_INVALID_ARG, "device step mask: a diagonal tile of the newest chunk was not kept");
   }
   return HYAT_OK;
 }

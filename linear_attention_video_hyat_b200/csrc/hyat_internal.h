@@ -17,6 +17,7 @@ constexpr int kTile = 128;          // query / key tile edge (rows)
 // Device status word bits (workspace offset 0).
 constexpr uint32_t kStatusTimeout = 1u;     // a bounded wait gave up
 constexpr uint32_t kStatusBadTile = 2u;     // a tile descriptor failed its bounds check
+constexpr uint32_t kStatusBadMask = 4u;     // a device step mask lacks a diagonal tile
 
 // A work item: one query tile and the key tiles of its softmax window.
 struct WorkItem {
@@ -104,15 +105,6 @@ struct SegStateArgs {
 };
 cudaError_t launch_seg_state(const SegStateArgs& a, cudaStream_t s);
 
-// Streaming fold, second half: srest[bh] += sum over r of partial[bh][r] (fixed order, so the
-// result is deterministic), and the bf16 copy of S for the attention kernel.
-struct FoldReduceArgs {
-  const float* partial;       // [BH][parts][E]
-  float* srest;               // [BH][E]
-  uint16_t* srest_bf16;       // [BH][d][d]
-  int32_t BH, parts, d;
-};
-cudaError_t launch_fold_reduce(const FoldReduceArgs& a, cudaStream_t s);
 cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t s);
 
 struct ComplementArgs {
@@ -172,21 +164,37 @@ cudaError_t launch_attn_tc_redo(const AttnArgs& a, const int4* redo_items, int32
 std::vector<int4> build_single_items(const std::vector<WorkItem>& work, int32_t num_sms);
 bool attn_tc_supported(int d, int dtype);
 
-struct RingCopyArgs {
+// A streaming step's work between the fold's state kernel and the attention (stream_prep.cu):
+// fold reduce, ring copy (K turned by the fused RoPE), Q turned into a workspace copy, and the
+// step's layout, in one launch. Every argument is the same for steps of the same ring phase
+// once the window is full, so a captured step replays for each of them.
+struct StreamPrepArgs {
+  int32_t nb_fold, nb_kv, nb_q, nb_layout;    // block ranges (set by launch_stream_prep)
+  int32_t BH, L, d, elem_bytes;
+  // fold reduce (partial = null: this step folds nothing)
+  const float* partial;           // [BH][parts][E]
+  float* srest;                   // [BH][E]
+  uint16_t* srest_bf16;           // [BH][d][d]
+  int32_t parts;
+  // ring copy
   const void* k; const void* v;   // [BH][L][d]
   void* ring_k; void* ring_v;     // [BH][nslots][L][d]
-  int32_t BH, L, d, nslots, slot, elem_bytes;
-};
-cudaError_t launch_ring_copy(const RingCopyArgs& a, cudaStream_t s);
-
-struct StreamLayoutArgs {
+  int32_t nslots, slot;
+  // fused RoPE (half_t = 0: none): frame f of the chunk turns by min(p0 + f, cap - 1) * theta
+  const void* q;                  // [BH][L][d]
+  void* q_out;                    // null: Q is not turned (no fused RoPE)
+  int32_t half_t, chunk_frames, tokens_per_frame, p0, cap;
+  double theta[64];               // base^(-2i / t_dims), i < half_t
+  // layout
   const uint8_t* mask;            // [mask_heads][nqt][nkt] (device)
   WorkItem* work;                 // [BH][nqt]
-  Entry* entries;                 // [BH][nqt][cap]
-  int32_t BH, H, mask_heads, nqt, nkt, cap, L, nwc;
+  Entry* entries;                 // [BH][nqt][cap_entries]
+  uint32_t* status;               // kStatusBadMask if a diagonal tile of the newest chunk is off
+  int32_t H, mask_heads, nqt, nkt, cap_entries, nwc;
   int32_t n_sink_visible;         // visible chunks 0..n_sink_visible-1 sit in slots nwc + c
-  int32_t first_window;           // the following visible chunks c >= first_window: slot c % nwc
+  int32_t first_window_mod;       // first window chunk mod nwc: window chunk w sits in slot
+                                  // (first_window_mod + w - n_sink_visible) % nwc
 };
-cudaError_t launch_stream_layout(const StreamLayoutArgs& a, cudaStream_t s);
+cudaError_t launch_stream_prep(StreamPrepArgs a, int num_sms, cudaStream_t s);
 
 }  // namespace hyat

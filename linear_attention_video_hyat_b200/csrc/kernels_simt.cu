@@ -1,8 +1,8 @@
 // CUDA-core kernels of libhyat: segment states, complement reduction, state
-// transpose, streaming ring copy and layout, and the fp32 hybrid-attention
-// kernel. The fp32 workload runs entirely here (the tensor cores have no fp32
-// operand kind, and tf32 is too coarse for a 1e-5 bound); the bf16 path uses
-// the tensor-core attention kernel and these kernels for its linear state.
+// transpose, and the fp32 hybrid-attention kernel. The fp32 workload runs
+// entirely here (the tensor cores have no fp32 operand kind, and tf32 is too
+// coarse for a 1e-5 bound); the bf16 path uses the tensor-core attention kernel
+// and these kernels for its linear state.
 //
 // Linear-state formation follows Hybrid Forcing, Section 2.A ("Hybrid
 // Attention": evicted key/value states aggregated into a compact state) and
@@ -170,71 +170,6 @@ __global__ void state_to_bf16_kernel(const float* __restrict__ s, uint16_t* __re
     const __nv_bfloat16 h = __float2bfloat16_rn(s[g * (dd + d) + e]);
     out[i] = *reinterpret_cast<const uint16_t*>(&h);
   }
-}
-
-// srest[bh] += sum_r partial[bh][r], in order r = 0, 1, ...; then bf16(S) for the attention
-// kernel. One thread per 4 consecutive floats of a state.
-__global__ void fold_reduce_kernel(FoldReduceArgs a) {
-  const int64_t E4 = (static_cast<int64_t>(a.d) * a.d + a.d) / 4, dd4 = static_cast<int64_t>(a.d) * a.d / 4;
-  const int64_t total = E4 * a.BH;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t bh = i / E4, e4 = i % E4;
-    float4* dst = reinterpret_cast<float4*>(a.srest) + bh * E4 + e4;
-    float4 acc = *dst;
-    const float4* src = reinterpret_cast<const float4*>(a.partial) + bh * a.parts * E4 + e4;
-    for (int r = 0; r < a.parts; ++r) {
-      const float4 v = src[r * E4];
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    *dst = acc;
-    if (e4 < dd4) {
-      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-      uint2 w;
-      w.x = *reinterpret_cast<const uint32_t*>(&lo);
-      w.y = *reinterpret_cast<const uint32_t*>(&hi);
-      reinterpret_cast<uint2*>(a.srest_bf16)[bh * dd4 + e4] = w;
-    }
-  }
-}
-
-// new chunk K/V -> ring slot, 16-byte vectors
-__global__ void ring_copy_kernel(RingCopyArgs a) {
-  const int64_t row_vecs = static_cast<int64_t>(a.L) * a.d * a.elem_bytes / 16;
-  const int64_t total = row_vecs * a.BH;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t bh = i / row_vecs, off = i % row_vecs;
-    const int64_t dst = (bh * a.nslots + a.slot) * row_vecs + off;
-    reinterpret_cast<uint4*>(a.ring_k)[dst] = reinterpret_cast<const uint4*>(a.k)[i];
-    reinterpret_cast<uint4*>(a.ring_v)[dst] = reinterpret_cast<const uint4*>(a.v)[i];
-  }
-}
-
-// per-step stream layout: one warp per (bh, query tile) compacts its mask row
-__global__ void stream_layout_kernel(StreamLayoutArgs a) {
-  const int lane = threadIdx.x;
-  const int bh = blockIdx.x / a.nqt, i = blockIdx.x % a.nqt;
-  const int hm = a.mask_heads == 1 ? 0 : bh % a.H;
-  const uint8_t* row = a.mask + (static_cast<int64_t>(hm) * a.nqt + i) * a.nkt;
-  const int64_t base = (static_cast<int64_t>(bh) * a.nqt + i) * a.cap;
-  int count = 0;
-  for (int kt0 = 0; kt0 < a.nkt; kt0 += 32) {
-    const int kt = kt0 + lane;
-    const bool keep = kt < a.nkt && row[kt] != 0;
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int pos = count + __popc(bal & ((1u << lane) - 1u));
-      const int w = kt / a.nqt, t = kt % a.nqt;
-      const int slot = w < a.n_sink_visible ? a.nwc + w : (a.first_window + w - a.n_sink_visible) % a.nwc;
-      a.entries[base + pos] = Entry{slot * a.L + t * kTile, min(kTile, a.L - t * kTile)};
-    }
-    count += __popc(bal);
-  }
-  if (lane == 0)
-    a.work[static_cast<int64_t>(bh) * a.nqt + i] =
-        WorkItem{bh, i * kTile, min(kTile, a.L - i * kTile), 0, static_cast<int32_t>(base),
-                 static_cast<int32_t>(base + count), 0, 0};
 }
 
 // --------------------------------------------------------------------------
@@ -476,28 +411,6 @@ cudaError_t launch_state_to_bf16(const float* srest, uint16_t* out, int64_t n_gr
 cudaError_t launch_attn_simt(const AttnArgs& a, cudaStream_t s) {
   if (a.dtype == HYAT_F32) return a.d == 64 ? launch_attn_simt_t<float, 64>(a, s) : launch_attn_simt_t<float, 128>(a, s);
   return a.d == 64 ? launch_attn_simt_t<__nv_bfloat16, 64>(a, s) : launch_attn_simt_t<__nv_bfloat16, 128>(a, s);
-}
-
-cudaError_t launch_fold_reduce(const FoldReduceArgs& a, cudaStream_t s) {
-  const int64_t total = (static_cast<int64_t>(a.d) * a.d + a.d) / 4 * a.BH;
-  if (total == 0) return cudaSuccess;
-  if (a.d % 4 != 0) return cudaErrorInvalidValue;
-  const int blocks = static_cast<int>((total + 255) / 256 < 2048 ? (total + 255) / 256 : 2048);
-  fold_reduce_kernel<<<blocks, 256, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_ring_copy(const RingCopyArgs& a, cudaStream_t s) {
-  const int64_t total = static_cast<int64_t>(a.L) * a.d * a.elem_bytes / 16 * a.BH;
-  if (total == 0) return cudaSuccess;
-  const int blocks = static_cast<int>((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
-  ring_copy_kernel<<<blocks, 256, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_stream_layout(const StreamLayoutArgs& a, cudaStream_t s) {
-  stream_layout_kernel<<<a.BH * a.nqt, 32, 0, s>>>(a);
-  return cudaGetLastError();
 }
 
 }  // namespace hyat

@@ -81,6 +81,14 @@ std::string validate_config(const hyat_config& c) {
     default:
       return "unknown mode";
   }
+  if (c.rope_t_dims != 0) {
+    if (c.mode != HYAT_MODE_STREAM) return "the fused temporal RoPE is a STREAM option";
+    if (c.rope_t_dims < 0 || c.rope_t_dims > c.d || c.rope_t_dims % 2 != 0)
+      return "rope_t_dims must be even and at most d";
+    if (c.rope_cap < 1) return "rope_cap must be >= 1";
+    if (!(c.rope_base >= 0.0f) || std::isinf(c.rope_base)) return "rope_base must be finite and >= 0";
+    if (static_cast<int64_t>(c.chunk_frames) * c.rope_t_dims > 8192) return "chunk_frames * rope_t_dims must be <= 8192";
+  }
   const int64_t n = rows_k(c) > rows_q(c) ? rows_k(c) : rows_q(c);
   if (n * c.d >= (int64_t(1) << 31)) return "rows * d per head must be < 2^31";
   if (static_cast<int64_t>(c.B) * c.H * n * c.d >= (int64_t(1) << 40)) return "tensor too large";

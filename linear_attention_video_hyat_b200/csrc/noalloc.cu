@@ -30,9 +30,11 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 int g_num_sms[kMaxDevices] = {};
+int g_major[kMaxDevices] = {};
 
-// Resolve the scratch address and SM count of the current device (once per device).
-cudaError_t scratch_for_current_device(void** addr, int* num_sms) {
+// Resolve the scratch address, SM count and compute-capability major of the current device
+// (once per device).
+cudaError_t scratch_for_current_device(void** addr, int* num_sms, int* major) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -42,14 +44,17 @@ cudaError_t scratch_for_current_device(void** addr, int* num_sms) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    int sms = 0;
+    int sms = 0, mj = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, dev);
     if (e != cudaSuccess) return e;
     g_scratch_addr[dev] = p;
     g_num_sms[dev] = sms;
+    g_major[dev] = mj;
   }
   *addr = g_scratch_addr[dev];
   *num_sms = g_num_sms[dev];
+  *major = g_major[dev];
   return cudaSuccess;
 }
 
@@ -67,13 +72,27 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   if (cfg->mode != HYAT_MODE_WINDOW && cfg->mode != HYAT_MODE_RADIAL) return HYAT_ERR_INVALID_ARG;
   for (const void* p : {q, k, v, static_cast<const void*>(o)})
     if (reinterpret_cast<uintptr_t>(p) & 15u) return HYAT_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The layout tables travel from pageable host vectors that die when this call returns; a
+  // captured copy would read them at replay. So the call refuses stream capture.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return HYAT_ERR_CUDA;
+  if (cap != cudaStreamCaptureStatusNone) return HYAT_ERR_UNSUPPORTED;
 
   Layout L;
   if (!build_layout(*cfg, nullptr, &L).empty()) return HYAT_ERR_INVALID_ARG;
-  std::vector<int4> pairs;   // chosen once the SM count is known; at most one per work item
   const int64_t BH = int64_t(cfg->B) * cfg->H;
   const int64_t E = int64_t(cfg->d) * cfg->d + cfg->d;
   const int64_t rows = rows_q(*cfg);
+  const int32_t nseg_pad = (L.nseg + 63) / 64 * 64;
+
+  void* base = nullptr;
+  int num_sms = 0, major = 0;
+  if (scratch_for_current_device(&base, &num_sms, &major) != cudaSuccess) return HYAT_ERR_CUDA;
+  // the same kernels as hyat_fwd_bidir on a handle of this configuration
+  const bool use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
+                      attn_tc_supported(cfg->d, cfg->dtype);
+  const bool use_gemm = use_tc && cfg->mode == HYAT_MODE_RADIAL && complement_tc_supported(cfg->d, L.nqg);
 
   // carve the static scratch
   size_t off = 0;
@@ -83,52 +102,72 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   const size_t o_entries = take(sizeof(Entry) * (L.entries.empty() ? 1 : L.entries.size()));
   const size_t o_pairs = take(sizeof(int4) * (L.work.empty() ? 1 : L.work.size()));
   const size_t o_cm = take(sizeof(float) * L.cm.size());
-  const size_t o_sseg = take(sizeof(float) * size_t(BH) * L.nseg * E);
+  const size_t o_cm_bf16 = use_gemm ? take(2 * size_t(L.cm_heads) * L.nqg * nseg_pad) : 0;
+  const size_t o_sseg = take(sizeof(float) * size_t(BH) * L.nseg * E);   // or its bf16 hi/lo parts
   const size_t o_srest = take(sizeof(float) * size_t(BH) * L.nqg * E);
   const size_t o_srest_bf16 = take(2 * size_t(BH) * L.nqg * cfg->d * cfg->d);
   if (off > kNoAllocScratchBytes) return HYAT_ERR_UNSUPPORTED;  // needs more than the static scratch
 
-  void* base = nullptr;
-  int num_sms = 0;
-  if (scratch_for_current_device(&base, &num_sms) != cudaSuccess) return HYAT_ERR_CUDA;
-  pairs = choose_pairs(L.work, num_sms);
+  const std::vector<int4> pairs = choose_pairs(L.work, num_sms);   // at most one per work item
+  std::vector<uint16_t> cmb;
+  if (use_gemm) {   // the 0/1 complement matrix in bf16 (exact), rows padded to 64 segments
+    cmb.assign(size_t(L.cm_heads) * L.nqg * nseg_pad, 0);
+    for (int32_t m = 0; m < L.cm_heads; ++m)
+      for (int32_t g = 0; g < L.nqg; ++g)
+        for (int32_t sg = 0; sg < L.nseg; ++sg)
+          if (L.cm[(size_t(m) * L.nqg + g) * L.nseg + sg] != 0.0f) cmb[(size_t(m) * L.nqg + g) * nseg_pad + sg] = 0x3F80;
+  }
   char* ws = static_cast<char*>(base);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   // layout tables: pageable host -> scratch (the copy has consumed the vectors when it returns);
   // the status word starts at zero on every call
   cudaError_t e = cudaMemsetAsync(ws + o_status, 0, 256, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(ws + o_work, L.work.data(), sizeof(WorkItem) * L.work.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !L.work.empty())
+    e = cudaMemcpyAsync(ws + o_work, L.work.data(), sizeof(WorkItem) * L.work.size(), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !L.entries.empty())
     e = cudaMemcpyAsync(ws + o_entries, L.entries.data(), sizeof(Entry) * L.entries.size(), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess && !pairs.empty())
     e = cudaMemcpyAsync(ws + o_pairs, pairs.data(), sizeof(int4) * pairs.size(), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess && !L.cm.empty())
     e = cudaMemcpyAsync(ws + o_cm, L.cm.data(), sizeof(float) * L.cm.size(), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && use_gemm)
+    e = cudaMemcpyAsync(ws + o_cm_bf16, cmb.data(), 2 * cmb.size(), cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return HYAT_ERR_CUDA;
 
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + o_status);
   SegStateArgs sa{};
   sa.k = k; sa.v = v; sa.rows_per_bh = rows;
   sa.BH = static_cast<int32_t>(BH); sa.d = cfg->d; sa.dtype = cfg->dtype; sa.phi = cfg->phi;
   sa.nseg = L.nseg; sa.seg_base = 0; sa.seg_stride = L.seg_stride; sa.seg_len = L.seg_len;
-  sa.out = reinterpret_cast<float*>(ws + o_sseg); sa.accumulate = 0;
-  if (launch_seg_state(sa, s) != cudaSuccess) return HYAT_ERR_CUDA;
+  sa.out = reinterpret_cast<float*>(ws + o_sseg); sa.accumulate = 0; sa.status = status;
+  if (use_gemm) {           // hi/lo bf16 parts for the tensor-core complement, in the same bytes
+    sa.out_hi = reinterpret_cast<uint16_t*>(ws + o_sseg);
+    sa.out_lo = sa.out_hi + size_t(BH) * L.nseg * E;
+  }
+  e = use_tc ? launch_seg_state_tc(sa, num_sms, s) : launch_seg_state(sa, s);
+  if (e != cudaSuccess) return HYAT_ERR_CUDA;
 
-  ComplementArgs ca{};
-  ca.sseg = sa.out; ca.cm = reinterpret_cast<const float*>(ws + o_cm);
-  ca.srest = reinterpret_cast<float*>(ws + o_srest);
-  ca.BH = static_cast<int32_t>(BH); ca.H = cfg->H; ca.cm_heads = L.cm_heads; ca.nseg = L.nseg; ca.nqg = L.nqg;
-  ca.E = static_cast<int32_t>(E);
-  ca.d = cfg->d;
-  int major = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
-    return HYAT_ERR_CUDA;
-  const bool use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
-                      attn_tc_supported(cfg->d, cfg->dtype);
-  ca.srest_bf16 = use_tc ? reinterpret_cast<uint16_t*>(ws + o_srest_bf16) : nullptr;
-  ca.write_f32_s = use_tc ? 0 : 1;
-  if (launch_complement(ca, s) != cudaSuccess) return HYAT_ERR_CUDA;
+  float* srest = reinterpret_cast<float*>(ws + o_srest);
+  uint16_t* srest_bf16 = reinterpret_cast<uint16_t*>(ws + o_srest_bf16);
+  if (use_gemm) {
+    ComplementTcArgs ga{};
+    ga.cm_bf16 = reinterpret_cast<const uint16_t*>(ws + o_cm_bf16);
+    ga.seg_hi = sa.out_hi; ga.seg_lo = sa.out_lo;
+    ga.srest = srest; ga.srest_bf16 = srest_bf16; ga.write_f32_s = 0;
+    ga.BH = static_cast<int32_t>(BH); ga.H = cfg->H; ga.mask_heads = L.cm_heads; ga.nqg = L.nqg; ga.nseg = L.nseg;
+    ga.nseg_pad = nseg_pad; ga.E = static_cast<int32_t>(E); ga.status = status;
+    e = launch_complement_tc(ga, num_sms, s);
+  } else {
+    ComplementArgs ca{};
+    ca.sseg = sa.out; ca.cm = reinterpret_cast<const float*>(ws + o_cm);
+    ca.srest = srest;
+    ca.srest_bf16 = use_tc ? srest_bf16 : nullptr;
+    ca.write_f32_s = use_tc ? 0 : 1;        // the tensor-core path reads S as bf16, z as fp32
+    ca.BH = static_cast<int32_t>(BH); ca.H = cfg->H; ca.cm_heads = L.cm_heads; ca.nseg = L.nseg; ca.nqg = L.nqg;
+    ca.E = static_cast<int32_t>(E); ca.d = cfg->d;
+    e = launch_complement(ca, s);
+  }
+  if (e != cudaSuccess) return HYAT_ERR_CUDA;
 
   AttnArgs a{};
   a.q = q; a.k = k; a.v = v; a.o = o;
@@ -138,18 +177,13 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   a.entries = reinterpret_cast<const Entry*>(ws + o_entries);
   a.pairs = reinterpret_cast<const int4*>(ws + o_pairs);
   a.n_pairs = static_cast<int32_t>(pairs.size());
-  a.srest = ca.srest;
-  a.srest_bf16 = reinterpret_cast<const uint16_t*>(ws + o_srest_bf16);
+  a.srest = srest;
+  a.srest_bf16 = srest_bf16;
   a.nqg = L.nqg; a.d = cfg->d; a.dtype = cfg->dtype; a.BH = static_cast<int32_t>(BH);
   const float scale = cfg->scale > 0.0f ? cfg->scale : 1.0f / sqrtf(float(cfg->d));
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.status = reinterpret_cast<uint32_t*>(ws + o_status);
+  a.status = status;
   a.phi = cfg->phi;
-
-  if (use_tc) {
-    if (launch_attn_tc(a, num_sms, s) != cudaSuccess) return HYAT_ERR_CUDA;
-  } else {
-    if (launch_attn_simt(a, s) != cudaSuccess) return HYAT_ERR_CUDA;
-  }
-  return HYAT_OK;
+  e = use_tc ? launch_attn_tc(a, num_sms, s) : launch_attn_simt(a, s);
+  return e == cudaSuccess ? HYAT_OK : HYAT_ERR_CUDA;
 }

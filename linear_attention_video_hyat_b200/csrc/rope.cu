@@ -16,61 +16,25 @@
 #include <cstdint>
 
 #include "hyat.h"
+#include "rope_common.cuh"
 
 namespace hyat {
 namespace {
 
 constexpr int kRopeRows = 128;    // tokens of one (b, h) per block
 constexpr int kRopeThreads = 256;
-constexpr int kMaxPairs = 64;     // d <= 128
 constexpr int kBatch = 4;         // rows a thread loads before it stores (memory parallelism)
 
 struct RopeArgs {
   const void* x;
   void* y;
   int32_t n_tokens, d, tokens_per_frame, first_frame, ref_frame, cap, half_t;
-  double theta[kMaxPairs];        // base^(-2i / t_dims), i < half_t
-};
-
-template <typename T>
-struct Lanes;
-template <>
-struct Lanes<float> {
-  static constexpr int kElems = 4;
-  __device__ static void to_f32(const uint4& v, float (&f)[4]) {
-    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
-    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
-  }
-  __device__ static uint4 from_f32(const float (&f)[4]) {
-    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
-  }
-};
-template <>
-struct Lanes<__nv_bfloat16> {
-  static constexpr int kElems = 8;
-  __device__ static void to_f32(const uint4& v, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
-      f[2 * e] = t.x;
-      f[2 * e + 1] = t.y;
-    }
-  }
-  __device__ static uint4 from_f32(const float (&f)[8]) {
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const __nv_bfloat162 t = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
-      w[e] = *reinterpret_cast<const uint32_t*>(&t);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-  }
+  double theta[kRopeMaxPairs];        // base^(-2i / t_dims), i < half_t
 };
 
 template <typename T>
 __global__ void __launch_bounds__(kRopeThreads) rope_temporal_kernel(const RopeArgs a) {
-  constexpr int E = Lanes<T>::kElems, P = E / 2;
+  constexpr int E = RopeLanes<T>::kElems, P = E / 2;
   const int cols = a.d / E;                        // 16-byte columns per row
   const int tx = threadIdx.x % cols, ty = threadIdx.x / cols, ny = kRopeThreads / cols;
   const int pair0 = tx * P;                        // first pair of this thread's column
@@ -103,26 +67,15 @@ __global__ void __launch_bounds__(kRopeThreads) rope_temporal_kernel(const RopeA
         if (p != cur_p) {
           cur_p = p;
 #pragma unroll
-          for (int k = 0; k < P; ++k) {
-            if (pair0 + k < a.half_t) {
-              double sd, cd;
-              sincos(static_cast<double>(p) * a.theta[pair0 + k], &sd, &cd);
-              c[k] = static_cast<float>(cd);
-              s[k] = static_cast<float>(sd);
-            }
-          }
+          for (int k = 0; k < P; ++k)
+            if (pair0 + k < a.half_t) rope_cos_sin(p, a.theta[pair0 + k], &c[k], &s[k]);
         }
         float f[E];
-        Lanes<T>::to_f32(v[b], f);
+        RopeLanes<T>::to_f32(v[b], f);
 #pragma unroll
-        for (int k = 0; k < P; ++k) {
-          if (pair0 + k < a.half_t) {
-            const float x0 = f[2 * k], x1 = f[2 * k + 1];
-            f[2 * k] = x0 * c[k] - x1 * s[k];
-            f[2 * k + 1] = x0 * s[k] + x1 * c[k];
-          }
-        }
-        v[b] = Lanes<T>::from_f32(f);
+        for (int k = 0; k < P; ++k)
+          if (pair0 + k < a.half_t) rope_turn(f[2 * k], f[2 * k + 1], c[k], s[k]);
+        v[b] = RopeLanes<T>::from_f32(f);
       }
       dst[(base_row + r) * cols + tx] = v[b];
     }

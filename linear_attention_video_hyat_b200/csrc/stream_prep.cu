@@ -1,0 +1,178 @@
+// The work of a streaming step between the fold's state kernel and the attention kernel, in one
+// launch (Long-Horizon Streaming Video Generation via Hybrid Attention with Decoupled
+// Distillation, Section 2.A: frames that leave the window are folded into the linear state,
+// the window keeps the latest frames for block-sparse softmax attention; Section 2.C: the
+// temporal RoPE index is a capped offset). Four independent jobs, each on its own range of
+// blocks:
+//   * fold reduce: S, z += the fold's partial states, summed in a fixed order (so a run is
+//     bit-reproducible), and the bf16 copy of S that the attention's linear-term MMA reads;
+//   * ring copy: the chunk's K and V into its ring slot, 16-byte vectors; with the fused RoPE,
+//     K is turned on its way in (the copy reads and writes every K vector anyway);
+//   * Q rotation (fused RoPE only): Q turned into a workspace copy that the attention reads;
+//   * layout: one warp per (b, h, query tile) compacts its row of the step's tile mask into
+//     the key-tile list (ring rows), and checks that the diagonal tile of the newest chunk is
+//     kept.
+// The kernel streams its bytes once (HBM-bound); it waits for the fold's partial states (and
+// for the fold to have read the ring slot it overwrites) with a programmatic-launch wait, and
+// lets the attention kernel start its prologue early.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "hyat_internal.h"
+#include "rope_common.cuh"
+
+namespace hyat {
+namespace {
+
+constexpr int kPrepThreads = 256;
+
+template <typename T>
+__device__ __forceinline__ void turn_vector(uint4& v, int col, int half_t, const float2* cs) {
+  constexpr int E = RopeLanes<T>::kElems, P = E / 2;
+  const int pair0 = col * P;
+  if (pair0 >= half_t) return;
+  float f[E];
+  RopeLanes<T>::to_f32(v, f);
+#pragma unroll
+  for (int k = 0; k < P; ++k)
+    if (pair0 + k < half_t) rope_turn(f[2 * k], f[2 * k + 1], cs[pair0 + k].x, cs[pair0 + k].y);
+  v = RopeLanes<T>::from_f32(f);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPrepThreads) stream_prep_kernel(const StreamPrepArgs a) {
+  extern __shared__ float2 cs_table[];            // [chunk frame][pair]: (cos, sin)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  constexpr int E = RopeLanes<T>::kElems;
+  const int cols = a.d / E;                       // 16-byte vectors per row
+  const int64_t row_vecs = static_cast<int64_t>(a.L) * cols;
+  int b = blockIdx.x;
+
+  // ---- fold reduce: srest[bh] += sum_r partial[bh][r], r in order; bf16 copy of S
+  if (b < a.nb_fold) {
+    const int64_t E4 = (static_cast<int64_t>(a.d) * a.d + a.d) / 4, dd4 = static_cast<int64_t>(a.d) * a.d / 4;
+    for (int64_t i = static_cast<int64_t>(b) * kPrepThreads + threadIdx.x; i < E4 * a.BH;
+         i += static_cast<int64_t>(a.nb_fold) * kPrepThreads) {
+      const int64_t bh = i / E4, e4 = i % E4;
+      float4* dst = reinterpret_cast<float4*>(a.srest) + bh * E4 + e4;
+      float4 acc = *dst;
+      const float4* src = reinterpret_cast<const float4*>(a.partial) + bh * a.parts * E4 + e4;
+      for (int r = 0; r < a.parts; ++r) {
+        const float4 v = src[r * E4];
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      *dst = acc;
+      if (e4 < dd4) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&lo);
+        w.y = *reinterpret_cast<const uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(a.srest_bf16)[bh * dd4 + e4] = w;
+      }
+    }
+    return;
+  }
+  b -= a.nb_fold;
+
+  // ---- K, V into the ring (K turned), or Q turned into its workspace copy
+  const bool is_kv = b < a.nb_kv;
+  if (is_kv || b < a.nb_kv + a.nb_q) {
+    const int nb = is_kv ? a.nb_kv : a.nb_q;
+    const int bb = is_kv ? b : b - a.nb_kv;
+    const bool turn = a.half_t > 0;
+    if (turn) {
+      // (cos, sin) of every (chunk frame, pair): frame f of the chunk sits at the capped
+      // offset min(p0 + f, cap - 1) from the reference frame
+      for (int i = threadIdx.x; i < a.chunk_frames * a.half_t; i += kPrepThreads) {
+        const int f = i / a.half_t, pr = i % a.half_t;
+        const int p = min(a.p0 + f, a.cap - 1);
+        float c, s;
+        rope_cos_sin(p, a.theta[pr], &c, &s);
+        cs_table[i] = make_float2(c, s);
+      }
+      __syncthreads();
+    }
+    const int64_t total = row_vecs * a.BH;
+    for (int64_t i = static_cast<int64_t>(bb) * kPrepThreads + threadIdx.x; i < total;
+         i += static_cast<int64_t>(nb) * kPrepThreads) {
+      const int64_t bh = i / row_vecs, off = i % row_vecs;
+      const int col = static_cast<int>(off % cols);
+      const float2* cs = cs_table + (static_cast<int>(off / cols) / a.tokens_per_frame) * a.half_t;
+      if (is_kv) {
+        const int64_t dst = (bh * a.nslots + a.slot) * row_vecs + off;
+        uint4 kv = reinterpret_cast<const uint4*>(a.k)[i];
+        const uint4 vv = reinterpret_cast<const uint4*>(a.v)[i];
+        if (turn) turn_vector<T>(kv, col, a.half_t, cs);
+        reinterpret_cast<uint4*>(a.ring_k)[dst] = kv;
+        reinterpret_cast<uint4*>(a.ring_v)[dst] = vv;
+      } else {
+        uint4 qv = reinterpret_cast<const uint4*>(a.q)[i];
+        turn_vector<T>(qv, col, a.half_t, cs);
+        reinterpret_cast<uint4*>(a.q_out)[i] = qv;
+      }
+    }
+    return;
+  }
+  b -= a.nb_kv + a.nb_q;
+
+  // ---- layout: one warp per (bh, query tile)
+  const int lane = threadIdx.x & 31;
+  const int item = b * (kPrepThreads / 32) + (threadIdx.x >> 5);
+  if (item >= a.BH * a.nqt) return;
+  const int bh = item / a.nqt, i = item % a.nqt;
+  const int hm = a.mask_heads == 1 ? 0 : bh % a.H;
+  const uint8_t* row = a.mask + (static_cast<int64_t>(hm) * a.nqt + i) * a.nkt;
+  const int64_t base = static_cast<int64_t>(item) * a.cap_entries;
+  int count = 0;
+  for (int kt0 = 0; kt0 < a.nkt; kt0 += 32) {
+    const int kt = kt0 + lane;
+    const bool keep = kt < a.nkt && row[kt] != 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = count + __popc(bal & ((1u << lane) - 1u));
+      const int w = kt / a.nqt, t = kt % a.nqt;
+      const int slot = w < a.n_sink_visible ? a.nwc + w : (a.first_window_mod + w - a.n_sink_visible) % a.nwc;
+      a.entries[base + pos] = Entry{slot * a.L + t * kTile, min(kTile, a.L - t * kTile)};
+    }
+    count += __popc(bal);
+  }
+  if (lane == 0) {
+    if (row[a.nkt - a.nqt + i] == 0) atomicOr(a.status, kStatusBadMask);
+    a.work[item] = WorkItem{bh, i * kTile, min(kTile, a.L - i * kTile), 0, static_cast<int32_t>(base),
+                            static_cast<int32_t>(base + count), 0, 0};
+  }
+}
+
+int blocks_for(int64_t n, int cap) {
+  const int64_t b = (n + kPrepThreads - 1) / kPrepThreads;
+  return static_cast<int>(b < cap ? b : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_stream_prep(StreamPrepArgs a, int num_sms, cudaStream_t s) {
+  const int E = a.elem_bytes == 4 ? 4 : 8;
+  if (a.d % E != 0 || (a.half_t > 0 && a.chunk_frames * a.half_t * 8 > 48 * 1024)) return cudaErrorInvalidValue;
+  const int64_t vecs = static_cast<int64_t>(a.L) * (a.d / E) * a.BH;
+  a.nb_fold = a.partial ? blocks_for((static_cast<int64_t>(a.d) * a.d + a.d) / 4 * a.BH, 2 * num_sms) : 0;
+  a.nb_kv = blocks_for(vecs, 8 * num_sms);
+  a.nb_q = a.q_out ? blocks_for(vecs, 4 * num_sms) : 0;
+  a.nb_layout = (a.BH * a.nqt + kPrepThreads / 32 - 1) / (kPrepThreads / 32);
+  const int grid = a.nb_fold + a.nb_kv + a.nb_q + a.nb_layout;
+  const size_t smem = a.half_t > 0 ? sizeof(float2) * a.chunk_frames * a.half_t : 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPrepThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return a.elem_bytes == 4 ? cudaLaunchKernelEx(&cfg, stream_prep_kernel<float>, a)
+                           : cudaLaunchKernelEx(&cfg, stream_prep_kernel<__nv_bfloat16>, a);
+}
+
+}  // namespace hyat

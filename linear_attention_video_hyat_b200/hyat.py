@@ -24,7 +24,7 @@ FLAG_SIMT = 1
 FLAG_TEST_DEVICE_TIMEOUT = 2
 FLAG_SINGLE_TILE = 4
 TILE = 128
-KERNEL_KINDS = ("state", "complement", "attention", "fold_ring", "layout_prep")
+KERNEL_KINDS = ("state", "complement", "attention", "fold", "prep")
 
 _MODES = {"window": MODE_WINDOW, "blockmask": MODE_BLOCKMASK, "radial": MODE_RADIAL, "stream": MODE_STREAM,
           "lvsa": MODE_BLOCKMASK}   # LVSA: a block mask from lvsa_mask()
@@ -34,7 +34,8 @@ EXPORTED = (
     "hyat_destroy", "hyat_last_error", "hyat_status_string", "hyat_plan_layout", "hyat_radial_mask",
     "hyat_stream_plan", "hyat_stream_state_bytes", "hyat_stream_get_state", "hyat_stream_set_state",
     "hyat_set_profiling", "hyat_kernel_times", "hyat_fwd_bidir_noalloc", "hyat_fwd_stream_denoise",
-    "hyat_lvsa_mask", "hyat_rope_temporal",
+    "hyat_lvsa_mask", "hyat_rope_temporal", "hyat_fwd_stream_step_dev", "hyat_fwd_stream_step_graph",
+    "hyat_stream_get_layout",
 )
 
 
@@ -52,6 +53,7 @@ class Config(ctypes.Structure):
         ("window_frames", ctypes.c_int32), ("mode", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("phi", ctypes.c_int32), ("mask_heads", ctypes.c_int32), ("flags", ctypes.c_uint32),
         ("scale", ctypes.c_float), ("sink_frames", ctypes.c_int32),
+        ("rope_t_dims", ctypes.c_int32), ("rope_cap", ctypes.c_int32), ("rope_base", ctypes.c_float),
     ]
 
 
@@ -68,6 +70,9 @@ def _load():
         "hyat_fwd_bidir": (ctypes.c_int, [P, P, P, P, P, P]),
         "hyat_fwd_stream_step": (ctypes.c_int, [P, P, P, P, P, P, P]),
         "hyat_fwd_stream_denoise": (ctypes.c_int, [P, P, P, P, P, P, P]),
+        "hyat_fwd_stream_step_dev": (ctypes.c_int, [P, P, P, P, P, P, P]),
+        "hyat_fwd_stream_step_graph": (ctypes.c_int, [P, P, P, P, P, P, P]),
+        "hyat_stream_get_layout": (ctypes.c_int, [P, P, S, P, S, P, S, ctypes.POINTER(I64)]),
         "hyat_sync": (ctypes.c_int, [P]),
         "hyat_destroy": (ctypes.c_int, [P]),
         "hyat_last_error": (ctypes.c_char_p, [P]),
@@ -99,18 +104,22 @@ PHI = {"elu1": 0, "relu": 1, "exp": 2}   # hyat_phi
 
 def make_config(mode, B, H, d, tokens_per_frame, n_frames=0, chunk_frames=1, halo_frames=0,
                 window_frames=0, dtype=BF16, mask_heads=1, flags=0, scale=0.0, phi="elu1",
-                sink_frames=0) -> Config:
+                sink_frames=0, rope=None) -> Config:
+    """rope: None, or {"t_dims", "cap", "base"} for the capped temporal RoPE fused into a STREAM
+    handle's steps (see hyat_config.rope_t_dims)."""
     m = _MODES[mode] if isinstance(mode, str) else int(mode)
     dt = {"f32": F32, "bf16": BF16}.get(dtype, dtype) if isinstance(dtype, str) else int(dtype)
     ph = PHI[phi] if isinstance(phi, str) else int(phi)
     return Config(B, H, d, tokens_per_frame, n_frames, chunk_frames, halo_frames, window_frames,
-                  m, dt, ph, mask_heads, flags, float(scale), int(sink_frames))
+                  m, dt, ph, mask_heads, flags, float(scale), int(sink_frames),
+                  int(rope["t_dims"]) if rope else 0, int(rope["cap"]) if rope else 0,
+                  float(rope.get("base", 0.0)) if rope else 0.0)
 
 
-def config_from_workload(w, flags=0, mask_heads=1) -> Config:
+def config_from_workload(w, flags=0, mask_heads=1, rope=None) -> Config:
     return make_config(w.mode, w.B, w.H, w.d, w.tokens_per_frame, w.n_frames, w.chunk_frames,
                        w.halo_frames, w.window_frames, w.dtype, mask_heads=mask_heads, flags=flags,
-                       phi=getattr(w, "phi", "elu1"), sink_frames=getattr(w, "sink_frames", 0))
+                       phi=getattr(w, "phi", "elu1"), sink_frames=getattr(w, "sink_frames", 0), rope=rope)
 
 
 def _check(status, handle=None):
@@ -254,6 +263,38 @@ class Hyat:
     def stream_step(self, q, k, v, mask=None, out=None, stream=None):
         """The current chunk's final call: attend, then keep its K, V and advance."""
         return self._stream_call(lib.hyat_fwd_stream_step, q, k, v, mask, out, stream)
+
+    def stream_step_dev(self, q, k, v, mask=None, out=None, stream=None, graph=False):
+        """stream_step with the mask as a uint8 CUDA tensor (None: every tile kept); graph=True
+        replays steady steps from CUDA graphs captured by the library."""
+        c = self.cfg
+        L = c.chunk_frames * c.tokens_per_frame
+        for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+            self._check_t(t, nm, L)
+        out = torch.empty_like(q) if out is None else out
+        self._check_t(out, "out", L)
+        if mask is not None and (mask.device.type != "cuda" or mask.dtype != torch.uint8 or not mask.is_contiguous()):
+            raise ValueError("mask: need a contiguous uint8 CUDA tensor")
+        s = torch.cuda.current_stream(q.device) if stream is None else stream
+        fn = lib.hyat_fwd_stream_step_graph if graph else lib.hyat_fwd_stream_step_dev
+        _check(fn(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                  None if mask is None else mask.data_ptr(), s.cuda_stream), self.handle)
+        return out
+
+    def stream_layout(self):
+        """The layout the last streaming call built on the device: (work [n, 8], entries
+        [n, cap, 2], plan info of that step, step)."""
+        counts = (ctypes.c_int64 * 3)()
+        _check(lib.hyat_stream_get_layout(self.handle, None, 0, None, 0, None, 0, counts), self.handle)
+        n, ne = counts[0], counts[1]
+        c = self.cfg
+        slots = c.window_frames // c.chunk_frames + c.sink_frames // c.chunk_frames
+        work = np.zeros((n, 8), np.int32)
+        ent = np.zeros((ne, 2), np.int32)
+        info = np.zeros(4 + slots, np.int32)
+        _check(lib.hyat_stream_get_layout(self.handle, work.ctypes.data, work.size, ent.ctypes.data, ent.size,
+                                          info.ctypes.data, info.size, counts), self.handle)
+        return work, ent.reshape(n, ne // max(n, 1), 2), info, int(counts[2])
 
     def stream_denoise(self, q, k, v, mask=None, out=None, stream=None):
         """A non-final call for the current chunk (one denoising step): attend with this

@@ -128,6 +128,26 @@ def test_invalid_configs_rejected(bad):
     assert hyat.workspace_bytes(cfg) == 0
 
 
+@pytest.mark.parametrize("rope,ok", [({"t_dims": 44, "cap": 21}, True), ({"t_dims": 128, "cap": 1, "base": 500.0}, True),
+                                     ({"t_dims": 43, "cap": 21}, False), ({"t_dims": 130, "cap": 21}, False),
+                                     ({"t_dims": 44, "cap": 0}, False), ({"t_dims": -2, "cap": 3}, False),
+                                     ({"t_dims": 44, "cap": 3, "base": -1.0}, False),
+                                     ({"t_dims": 44, "cap": 3, "base": float("inf")}, False)])
+def test_fused_rope_config_validation(rope, ok):
+    """The fused temporal RoPE is a STREAM option with an even band of at most d dimensions and
+    a cap of at least 1; its workspace adds the turned Q of one chunk."""
+    cfg = hyat.config_from_workload(wl.STREAM_HF, rope=rope)
+    plain = hyat.workspace_bytes(hyat.config_from_workload(wl.STREAM_HF))
+    n = hyat.workspace_bytes(cfg)
+    if ok:
+        q_bytes = wl.STREAM_HF.B * wl.STREAM_HF.H * wl.STREAM_HF.chunk_tokens * wl.STREAM_HF.d * 2
+        assert plain + q_bytes <= n <= plain + q_bytes + 256
+    else:
+        assert n == 0
+    # never on a bidirectional handle
+    assert hyat.workspace_bytes(hyat.config_from_workload(wl.WAN13B_BIDIR, rope={"t_dims": 44, "cap": 21})) == 0
+
+
 def test_workspace_sizes():
     for w in (wl.TINY_F32, wl.WAN13B_BIDIR, wl.WAN14B_BIDIR, wl.STREAM_HF, wl.RADIAL_84F):
         n = hyat.workspace_bytes(hyat.config_from_workload(w))
