@@ -65,6 +65,9 @@ def parse():
     p.add_argument("--rope", action="store_true",
                    help="streaming workload: the capped temporal RoPE of the chunk's Q and K fused "
                         "into each step (hyat_config.rope_t_dims)")
+    p.add_argument("--rope-standalone", action="store_true",
+                   help="streaming workload: the same RoPE as --rope, as two hyat_rope_temporal calls "
+                        "(Q, K) before each plain step (the unfused baseline of --rope)")
     p.add_argument("--graph", action="store_true",
                    help="streaming workload: device step masks, steady steps replayed from the "
                         "library's CUDA graphs (hyat_fwd_stream_step_graph)")
@@ -390,13 +393,37 @@ def bench_stream(a, w, rank, world, local):
     cfg = hyat.config_from_workload(w, mask_heads=w.H, rope=ROPE if a.rope else None)
     if a.graph:
         config["graph"] = "device masks; steady steps replayed from the library's CUDA graphs"
+    if a.rope or a.rope_standalone:
+        config["rope"] = dict(ROPE, ref="first frame of the oldest rolling-window chunk",
+                              path="fused into the step" if a.rope else "hyat_rope_temporal on Q and K, then the step")
+    nsink = w.sink_frames // w.chunk_frames
+    rope_events = []
+
+    def rope_standalone(q, k, s_, timed):
+        """The unfused RoPE of step s_: Q and K turned by their capped offsets from the first
+        frame of the oldest rolling-window chunk (the chunk's own while the window has none)."""
+        first_window = max(nsink, s_ - nwc + 1)
+        f0 = s_ * w.chunk_frames
+        ref = first_window * w.chunk_frames if s_ >= first_window else f0
+        if timed:
+            ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            ev[0].record(stream)
+        for x, y in ((q, qr), (k, kr)):
+            hyat.rope_temporal(x, w.tokens_per_frame, f0, ref, ROPE["cap"], ROPE["t_dims"], ROPE["base"], out=y)
+        if timed:
+            ev[1].record(stream)
+            rope_events.append(ev)
+        return qr, kr
     dev_in = [(q.to(dev), k.to(dev), v.to(dev), m, torch.from_numpy(np.ascontiguousarray(m)).to(dev))
               for q, k, v, m in inputs]
     od = torch.empty_like(dev_in[0][0])
+    qr, kr = torch.empty_like(od), torch.empty_like(od)      # the unfused RoPE's outputs
     stream = torch.cuda.current_stream(dev)
 
-    def step(h, x, m_host, s_, out):
+    def step(h, x, m_host, s_, out, timed=False):
         q, k, v, m, md = x
+        if a.rope_standalone:
+            q, k = rope_standalone(q, k, s_, timed)
         if s_ < nwc:          # the window is still filling: masks of the growing shape
             m = wl.gen_stream_step(w, s_, seed=w.seed + rank)[3]
             md = torch.from_numpy(np.ascontiguousarray(m)).to(dev)
@@ -405,10 +432,10 @@ def bench_stream(a, w, rank, world, local):
         else:
             h.stream_step(q, k, v, mask=m if m_host is None else m_host, out=out)
 
-    def run(h, steps, first):
+    def run(h, steps, first, timed=False):
         for i in range(steps):
             s_ = first + i
-            step(h, dev_in[s_ % n_dist], None, s_, od)
+            step(h, dev_in[s_ % n_dist], None, s_, od, timed)
 
     h = hyat.Hyat(cfg, device=dev)
     run(h, warm + n_dist * nwc, 0)        # warm-up (and, with --graph, one capture per phase and input set)
@@ -418,8 +445,9 @@ def bench_stream(a, w, rank, world, local):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local)
     host0 = time.perf_counter()
-    with ClockSampler(local) as clk:
+    with clk:
         t0.record(stream)
         run(h, a.steps, first)
         t1.record(stream)
@@ -431,12 +459,12 @@ def bench_stream(a, w, rank, world, local):
     h.set_profiling(True)        # per-launch events (graph replay is off while profiling)
     h.kernel_times()
     with ClockSampler(local) as clk2:
-        run(h, a.steps, first)
+        run(h, a.steps, first, timed=True)
         torch.cuda.synchronize(dev)
     first += a.steps
     kt = h.kernel_times()
     h.set_profiling(False)
-    launches = sum(n for _, n in kt.values())
+    launches = sum(n for _, n in kt.values()) + 2 * len(rope_events)
     value, tokens_per_s = job_throughput(mean_flops, w.B * w.chunk_tokens, ms, world)
     pk, pk_src = peaks()
     attn_ms = kt["attention"][0] / max(kt["attention"][1], 1)
@@ -457,6 +485,12 @@ def bench_stream(a, w, rank, world, local):
         pbytes = 4 * kv + (2 * kv if a.rope else 0)
         kernels["prep"]["algorithmic_bytes"] = pbytes
         kernels["prep"]["hbm_gbs"] = pbytes / (kernels["prep"]["ms_per_launch"] / 1e3) / 1e9
+    if rope_events:
+        r_ms = sum(e0.elapsed_time(e1) for e0, e1 in rope_events) / (2 * len(rope_events))
+        r_bytes = 2 * od.numel() * od.element_size()        # out of place: one read, one write
+        kernels["rope"] = {"ms_per_launch": r_ms, "launches": 2 * len(rope_events),
+                           "hbm_gbs": r_bytes / (r_ms / 1e3) / 1e9,
+                           "timing": "CUDA events around the Q and K calls of each step, pass 2"}
     config["host_ms_per_step"] = 1e3 * host_s / a.steps
 
     e2e = None
@@ -495,6 +529,8 @@ def bench_stream(a, w, rank, world, local):
                 if i >= 2:
                     stream.wait_event(out_free[b])
                 q, k, v = dbuf[b]
+                if a.rope_standalone:
+                    q, k = rope_standalone(q, k, counter[0], False)
                 if a.graph:
                     h.stream_step_dev(q, k, v, mask=dmask[b], out=dout[b], graph=True)
                 else:

@@ -25,6 +25,7 @@ namespace hyat {
 namespace {
 
 constexpr int kPrepThreads = 256;
+constexpr int kPrepUnroll = 4;        // vectors a thread moves at a time (memory parallelism)
 
 template <typename T>
 __device__ __forceinline__ void turn_vector(uint4& v, int col, int half_t, const float2* cs) {
@@ -94,22 +95,36 @@ __global__ void __launch_bounds__(kPrepThreads) stream_prep_kernel(const StreamP
       __syncthreads();
     }
     const int64_t total = row_vecs * a.BH;
-    for (int64_t i = static_cast<int64_t>(bb) * kPrepThreads + threadIdx.x; i < total;
-         i += static_cast<int64_t>(nb) * kPrepThreads) {
-      const int64_t bh = i / row_vecs, off = i % row_vecs;
-      const int col = static_cast<int>(off % cols);
-      const float2* cs = cs_table + (static_cast<int>(off / cols) / a.tokens_per_frame) * a.half_t;
-      if (is_kv) {
-        const int64_t dst = (bh * a.nslots + a.slot) * row_vecs + off;
-        uint4 kv = reinterpret_cast<const uint4*>(a.k)[i];
-        const uint4 vv = reinterpret_cast<const uint4*>(a.v)[i];
-        if (turn) turn_vector<T>(kv, col, a.half_t, cs);
-        reinterpret_cast<uint4*>(a.ring_k)[dst] = kv;
-        reinterpret_cast<uint4*>(a.ring_v)[dst] = vv;
-      } else {
-        uint4 qv = reinterpret_cast<const uint4*>(a.q)[i];
-        turn_vector<T>(qv, col, a.half_t, cs);
-        reinterpret_cast<uint4*>(a.q_out)[i] = qv;
+    const int64_t stride = static_cast<int64_t>(nb) * kPrepThreads;
+    // kPrepUnroll vectors per thread at a time: every load is issued before the first store
+    for (int64_t i0 = static_cast<int64_t>(bb) * kPrepThreads + threadIdx.x; i0 < total; i0 += stride * kPrepUnroll) {
+      uint4 x[kPrepUnroll], y[kPrepUnroll];
+#pragma unroll
+      for (int u = 0; u < kPrepUnroll; ++u) {
+        const int64_t i = i0 + u * stride;
+        if (i >= total) break;
+        if (is_kv) {
+          x[u] = reinterpret_cast<const uint4*>(a.k)[i];
+          y[u] = reinterpret_cast<const uint4*>(a.v)[i];
+        } else {
+          x[u] = reinterpret_cast<const uint4*>(a.q)[i];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPrepUnroll; ++u) {
+        const int64_t i = i0 + u * stride;
+        if (i >= total) break;
+        const int64_t bh = i / row_vecs, off = i % row_vecs;
+        const int col = static_cast<int>(off % cols);
+        const float2* cs = cs_table + (static_cast<int>(off / cols) / a.tokens_per_frame) * a.half_t;
+        if (turn) turn_vector<T>(x[u], col, a.half_t, cs);
+        if (is_kv) {
+          const int64_t dst = (bh * a.nslots + a.slot) * row_vecs + off;
+          reinterpret_cast<uint4*>(a.ring_k)[dst] = x[u];
+          reinterpret_cast<uint4*>(a.ring_v)[dst] = y[u];
+        } else {
+          reinterpret_cast<uint4*>(a.q_out)[i] = x[u];
+        }
       }
     }
     return;
@@ -156,8 +171,8 @@ cudaError_t launch_stream_prep(StreamPrepArgs a, int num_sms, cudaStream_t s) {
   if (a.d % E != 0 || (a.half_t > 0 && a.chunk_frames * a.half_t * 8 > 48 * 1024)) return cudaErrorInvalidValue;
   const int64_t vecs = static_cast<int64_t>(a.L) * (a.d / E) * a.BH;
   a.nb_fold = a.partial ? blocks_for((static_cast<int64_t>(a.d) * a.d + a.d) / 4 * a.BH, 2 * num_sms) : 0;
-  a.nb_kv = blocks_for(vecs, 8 * num_sms);
-  a.nb_q = a.q_out ? blocks_for(vecs, 4 * num_sms) : 0;
+  a.nb_kv = blocks_for((vecs + kPrepUnroll - 1) / kPrepUnroll, 8 * num_sms);
+  a.nb_q = a.q_out ? blocks_for((vecs + kPrepUnroll - 1) / kPrepUnroll, 4 * num_sms) : 0;
   a.nb_layout = (a.BH * a.nqt + kPrepThreads / 32 - 1) / (kPrepThreads / 32);
   const int grid = a.nb_fold + a.nb_kv + a.nb_q + a.nb_layout;
   const size_t smem = a.half_t > 0 ? sizeof(float2) * a.chunk_frames * a.half_t : 0;

@@ -448,8 +448,24 @@ def test_full_wan13b_bidir_sampled():
 
 
 @pytest.mark.slow
+def test_full_wan13b_bidir_whole_head():
+    """One head of the full Wan-1.3B layer, all 32760 rows, element by element against the
+    fp64 oracle (rows in blocks of one chunk)."""
+    w = wl.WAN13B_BIDIR
+    o, (q, k, v) = _bidir(w)
+    head = [7]
+    qs, ks, vs = q[:, head], k[:, head], v[:, head]
+    got = f64(o[:, head])
+    C = w.chunk_tokens
+    ref = np.concatenate([_window_ref(w, qs, ks, vs, rows=np.arange(c0, min(c0 + C, w.N)))
+                          for c0 in range(0, w.N, C)], axis=2)
+    assert ref.shape == got.shape == (1, 1, w.N, w.d)
+    assert_parity("bf16", got, ref, "wan1.3b head 7, every row")
+
+
+@pytest.mark.slow
 def test_full_wan14b_bidir_sampled():
-    got, ref = _bidir_sampled(wl.WAN14B_BIDIR, heads=[0, 17, 39], per_tile=1)
+    got, ref = _bidir_sampled(wl.WAN14B_BIDIR, heads=[0, 17, 39], per_tile=2)
     assert_parity("bf16", got, ref, "wan14b")
 
 
@@ -461,7 +477,7 @@ def test_full_radial_sampled():
 
 @pytest.mark.slow
 def test_full_lvsa_sampled():
-    got, ref = _bidir_sampled(wl.LVSA_126F, heads=[0, 7], per_tile=1)
+    got, ref = _bidir_sampled(wl.LVSA_126F, heads=[0, 7], per_tile=2)
     assert_parity("bf16", got, ref, "lvsa")
 
 
