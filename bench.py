@@ -36,7 +36,8 @@ from linear_attention_video_hyat_b200 import workloads as wl  # noqa: E402
 METRIC = "hybrid-attn effective TFLOP/s & tokens/s per layer; % of B200 BF16 TC peak"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["linear_attention_video_hyat_b200/csrc/attn_tc.cu"]
+# the attention call of the default schedule: the wide-softmax kernel and its redo pass
+KERNEL_SOURCES = ["linear_attention_video_hyat_b200/csrc/attn_tc_wide.cu", "linear_attention_video_hyat_b200/csrc/attn_tc.cu"]
 # the streaming bench's --rope step: a temporal band of 44 of the 128 head dimensions, the
 # index capped at 21 frames (the pages' example of a pretrained model's range), base 10000
 ROPE = {"t_dims": 44, "cap": 21, "base": 10000.0}
@@ -59,9 +60,11 @@ def parse():
     p.add_argument("--workload", default=wl.WAN13B_BIDIR.name, choices=sorted(wl.WORKLOADS))
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--schedule", choices=["pair", "single"], default="pair",
-                   help="tensor-core attention schedule of the bidirectional modes: a pair of query "
-                        "tiles per CTA (default) or one query tile per CTA (HYAT_FLAG_SINGLE_TILE)")
+    p.add_argument("--schedule", choices=["pair", "one-warp", "single"], default="pair",
+                   help="tensor-core attention schedule: a pair of query tiles per CTA with two softmax "
+                        "warps per row (default), the pair schedule with one softmax warp per row "
+                        "(HYAT_FLAG_PAIR_ONE_WARP), or one query tile per CTA (HYAT_FLAG_SINGLE_TILE; "
+                        "bidirectional modes)")
     p.add_argument("--rope", action="store_true",
                    help="streaming workload: the capped temporal RoPE of the chunk's Q and K fused "
                         "into each step (hyat_config.rope_t_dims)")
@@ -390,7 +393,9 @@ def bench_stream(a, w, rank, world, local):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    cfg = hyat.config_from_workload(w, mask_heads=w.H, rope=ROPE if a.rope else None)
+    cfg = hyat.config_from_workload(w, mask_heads=w.H, rope=ROPE if a.rope else None,
+                                    flags=hyat.FLAG_PAIR_ONE_WARP if a.schedule == "one-warp" else 0)
+    config["schedule"] = a.schedule
     if a.graph:
         config["graph"] = "device masks; steady steps replayed from the library's CUDA graphs"
     if a.rope or a.rope_standalone:
@@ -465,6 +470,8 @@ def bench_stream(a, w, rank, world, local):
     kt = h.kernel_times()
     h.set_profiling(False)
     launches = sum(n for _, n in kt.values()) + 2 * len(rope_events)
+    if a.schedule == "pair":
+        launches += kt["attention"][1]          # the attention kernel and its redo pass
     value, tokens_per_s = job_throughput(mean_flops, w.B * w.chunk_tokens, ms, world)
     pk, pk_src = peaks()
     attn_ms = kt["attention"][0] / max(kt["attention"][1], 1)
@@ -631,8 +638,8 @@ def main():
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     od = torch.empty_like(qd)
     single = a.schedule == "single"
-    h = hyat.Hyat(hyat.config_from_workload(w, flags=hyat.FLAG_SINGLE_TILE if single else 0), workload_mask(w),
-                  device=dev)
+    flags = {"single": hyat.FLAG_SINGLE_TILE, "one-warp": hyat.FLAG_PAIR_ONE_WARP}.get(a.schedule, 0)
+    h = hyat.Hyat(hyat.config_from_workload(w, flags=flags), workload_mask(w), device=dev)
     stream = torch.cuda.current_stream(dev)
     for _ in range(max(a.warmup, 3)):
         h.forward(qd, kd, vd, out=od)
@@ -664,8 +671,8 @@ def main():
     h.set_profiling(False)
     ms = max_over_ranks(ms, dev)
     launches = sum(n for _, n in kt.values())   # per-step launches x K (pass 2 mirrors pass 1)
-    if single:
-        launches += kt["attention"][1]          # each attention call is two kernels there (+ redo)
+    if a.schedule != "one-warp":
+        launches += kt["attention"][1]          # each attention call is two kernels (+ redo pass)
 
     value, tokens_per_s = job_throughput(counts["total_flops"], w.B * w.N, ms, world)
     pk, pk_src = peaks()

@@ -95,13 +95,18 @@ typedef enum {
  * 20 ms limit. The wait gives up, every role drains and frees TMEM, the status word is set,
  * and hyat_sync() returns HYAT_ERR_DEVICE_TIMEOUT; later calls on any handle work. */
 #define HYAT_FLAG_TEST_DEVICE_TIMEOUT 2u
-/* Schedule of the tensor-core attention in the bidirectional modes. By default a CTA runs a
- * pair of query tiles, one per softmax warpgroup (the streaming mode always does). With this
- * flag a CTA runs one query tile at a time: the two softmax warpgroups take alternate key
- * tiles and TMEM holds three S buffers. Both schedules give results within the same
- * tolerance; the second is currently the slower one on B200 and is kept for cross-checks and
- * timing. */
+/* Schedules of the tensor-core attention. By default a CTA runs a pair of query tiles (the
+ * streaming mode, a split pair of one tile), with two softmax warps per row, each taking 64 of
+ * a key tile's 128 keys, a fixed reference max of 0 and a redo list: query tiles whose row sums
+ * leave [2^-100, 2^100) (scores far above 0, or all far below 0 with no linear term) are
+ * recomputed right after by the one-warp-per-row pair kernel, which moves its reference max.
+ * HYAT_FLAG_SINGLE_TILE (bidirectional modes) runs one query tile per CTA at a time (three S
+ * buffers in TMEM; two softmax warpgroups on alternate key tiles), with the same redo list.
+ * HYAT_FLAG_PAIR_ONE_WARP runs the pair schedule with one softmax warp per row and an exact
+ * moving reference max (no redo list). All give results within the same tolerance; the
+ * default is the fastest on B200, the others are kept for cross-checks and timing. */
 #define HYAT_FLAG_SINGLE_TILE 4u
+#define HYAT_FLAG_PAIR_ONE_WARP 8u
 
 typedef struct {
   int32_t B, H, d;               /* d in {64, 128} */

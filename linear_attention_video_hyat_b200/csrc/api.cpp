@@ -62,6 +62,7 @@ Plan make_plan(const hyat_config& c, int64_t n_work, int64_t n_entries, const La
     p.mask = take(size_t(c.mask_heads) * nqt * nqt * slots);
     p.fold_partial = take(sizeof(float) * BH * fold_parts_cap(c) * E);
     if (c.rope_t_dims > 0) p.q_rot = take(size_t(BH * Lc * c.d * elem_bytes(c)));
+    p.redo = take(sizeof(int4) * std::max<int64_t>(n_work, 1));
   } else {
     p.cm = take(sizeof(float) * size_t(L.cm_heads) * L.nqg * L.nseg);
     if (c.mode == HYAT_MODE_BLOCKMASK || c.mode == HYAT_MODE_RADIAL)
@@ -118,6 +119,7 @@ struct hyat_ctx {
   // one query tile per CTA (attn_single_kernel) with its redo list; the two counters live in
   // the zeroed status region
   bool single = false;
+  bool wide = false;                 // two softmax warps per row (the default), with a redo list
   int4* d_redo = nullptr;
   int32_t* d_redo_count = nullptr;
   uint32_t* d_redo_done = nullptr;
@@ -229,6 +231,12 @@ AttnArgs attn_args(hyat_ctx* h, const void* q, const void* k, const void* v, voi
 hyat_status launch_attention(hyat_ctx* h, const AttnArgs& a, cudaStream_t s) {
   cudaError_t e = timed(h, K_ATTN, s, [&] {
     if (!h->use_tc) return launch_attn_simt(a, s);
+    if (h->wide) {
+      cudaError_t r = launch_attn_wide(a, h->d_redo_count, h->d_redo, static_cast<int32_t>(h->plan.n_work),
+                                       h->num_sms, s);
+      if (r == cudaSuccess) r = launch_attn_tc_redo(a, h->d_redo, h->d_redo_count, h->d_redo_done, h->num_sms, s);
+      return r;
+    }
     if (!h->single) return launch_attn_tc(a, h->num_sms, s);
     cudaError_t r = launch_attn_single(a, h->d_redo_count, h->d_redo, h->num_sms, s);
     if (r == cudaSuccess) r = launch_attn_tc_redo(a, h->d_redo, h->d_redo_count, h->d_redo_done, h->num_sms, s);
@@ -308,6 +316,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
     h->d_mask = reinterpret_cast<uint8_t*>(ws + h->plan.mask);
     h->d_fold_partial = reinterpret_cast<float*>(ws + h->plan.fold_partial);
     if (h->plan.q_rot) h->d_q_rot = ws + h->plan.q_rot;
+    h->d_redo = reinterpret_cast<int4*>(ws + h->plan.redo);
     if (cfg->rope_t_dims > 0) {
       const double base = cfg->rope_base > 0.0f ? static_cast<double>(cfg->rope_base) : 10000.0;
       for (int i = 0; i < cfg->rope_t_dims / 2; ++i) h->rope_theta[i] = std::pow(base, -2.0 * i / cfg->rope_t_dims);
@@ -332,6 +341,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   h->use_tc = cfg->dtype == HYAT_BF16 && !(cfg->flags & HYAT_FLAG_SIMT) && major == 10 &&
               attn_tc_supported(cfg->d, cfg->dtype);
   h->use_gemm = h->use_tc && h->d_cm_bf16 != nullptr && complement_tc_supported(cfg->d, h->lay.nqg);
+  h->wide = h->use_tc && !(cfg->flags & (HYAT_FLAG_SINGLE_TILE | HYAT_FLAG_PAIR_ONE_WARP));
   if (cfg->mode == HYAT_MODE_STREAM) {
     // token ranges of the fold: about one per SM, whole 64-token stages
     const int32_t Lc = stream_chunk_tokens(*cfg);

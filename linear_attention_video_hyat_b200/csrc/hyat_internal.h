@@ -159,6 +159,11 @@ cudaError_t launch_attn_tc(const AttnArgs& a, int num_sms, cudaStream_t s);
 // attn_tc_kernel, reading the count on the device and resetting it (and *done_count) to 0.
 cudaError_t launch_attn_single(const AttnArgs& a, int32_t* redo_count, int4* redo_items, int num_sms,
                                cudaStream_t s);
+// The pair schedule with two softmax warps per row (attn_tc_wide.cu): fixed reference max 0;
+// query tiles whose row sums leave [2^-100, 2^100) are appended to redo_items (at most
+// redo_cap) for launch_attn_tc_redo.
+cudaError_t launch_attn_wide(const AttnArgs& a, int32_t* redo_count, int4* redo_items, int32_t redo_cap, int num_sms,
+                             cudaStream_t s);
 cudaError_t launch_attn_tc_redo(const AttnArgs& a, const int4* redo_items, int32_t* redo_count,
                                 uint32_t* done_count, int num_sms, cudaStream_t s);
 std::vector<int4> build_single_items(const std::vector<WorkItem>& work, int32_t num_sms);

@@ -106,6 +106,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   const size_t o_sseg = take(sizeof(float) * size_t(BH) * L.nseg * E);   // or its bf16 hi/lo parts
   const size_t o_srest = take(sizeof(float) * size_t(BH) * L.nqg * E);
   const size_t o_srest_bf16 = take(2 * size_t(BH) * L.nqg * cfg->d * cfg->d);
+  const size_t o_redo = take(sizeof(int4) * (L.work.empty() ? 1 : L.work.size()));   // redo list
   if (off > kNoAllocScratchBytes) return HYAT_ERR_UNSUPPORTED;  // needs more than the static scratch
 
   const std::vector<int4> pairs = choose_pairs(L.work, num_sms);   // at most one per work item
@@ -120,7 +121,8 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   char* ws = static_cast<char*>(base);
 
   // layout tables: pageable host -> scratch (the copy has consumed the vectors when it returns);
-  // the status word starts at zero on every call
+  // the status region (status word, redo count and its finish counter) starts at zero on every
+  // call
   cudaError_t e = cudaMemsetAsync(ws + o_status, 0, 256, s);
   if (e == cudaSuccess && !L.work.empty())
     e = cudaMemcpyAsync(ws + o_work, L.work.data(), sizeof(WorkItem) * L.work.size(), cudaMemcpyHostToDevice, s);
@@ -184,6 +186,15 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = status;
   a.phi = cfg->phi;
-  e = use_tc ? launch_attn_tc(a, num_sms, s) : launch_attn_simt(a, s);
+  if (!use_tc) {
+    e = launch_attn_simt(a, s);
+  } else {
+    // the default schedule of hyat_fwd_bidir: two softmax warps per row, then the redo pass
+    int32_t* redo_count = reinterpret_cast<int32_t*>(ws + o_status + 64);
+    uint32_t* redo_done = reinterpret_cast<uint32_t*>(ws + o_status + 128);
+    int4* redo = reinterpret_cast<int4*>(ws + o_redo);
+    e = launch_attn_wide(a, redo_count, redo, static_cast<int32_t>(L.work.size()), num_sms, s);
+    if (e == cudaSuccess) e = launch_attn_tc_redo(a, redo, redo_count, redo_done, num_sms, s);
+  }
   return e == cudaSuccess ? HYAT_OK : HYAT_ERR_CUDA;
 }

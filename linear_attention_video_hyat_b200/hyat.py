@@ -23,6 +23,7 @@ MODE_WINDOW, MODE_BLOCKMASK, MODE_RADIAL, MODE_STREAM = range(4)
 FLAG_SIMT = 1
 FLAG_TEST_DEVICE_TIMEOUT = 2
 FLAG_SINGLE_TILE = 4
+FLAG_PAIR_ONE_WARP = 8
 TILE = 128
 KERNEL_KINDS = ("state", "complement", "attention", "fold", "prep")
 
