@@ -255,7 +255,8 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
       l = (lz[0] + lz[1]) + (lz[2] + lz[3]);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(p_full);   // one arrival per warp
     }
     if (p.test_timeout && !wait_warp(&sm->never, 0, sm, p.status)) return;
     for (int j = 0; j < n; ++j) {
@@ -319,7 +320,8 @@ __device__ __forceinline__ void softmax_role(Smem* sm, const TcParams& p, uint32
       l += rs;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(p_full);   // one arrival per warp
     }
     const uint32_t n_commits = static_cast<uint32_t>(n) + (lin ? 1u : 0u);
     if (!wait_warp(pv_done, (pv_phase + n_commits - 1) & 1u, sm, p.status)) return;
@@ -423,7 +425,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&sm->q_full[s], 1);
       mbar_init(&sm->q_empty[s], 1);
       mbar_init(&sm->s_full[s], 1);
-      mbar_init(&sm->p_full[s], 128);
+      mbar_init(&sm->p_full[s], 4);             // one arrival per softmax warp of the slot
       mbar_init(&sm->pv_done[s], 1);
     }
     mbar_init(&sm->xfull, 128);

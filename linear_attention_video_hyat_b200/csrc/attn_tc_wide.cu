@@ -222,7 +222,8 @@ __device__ __forceinline__ void softmax_wide(SmemW* sm, const WideParams& p, uin
       l = (lz[0] + lz[1]) + (lz[2] + lz[3]);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);        // one arrival per warp (its stores are done)
     }
     if (s == 0 && hf == 0 && p.test_timeout && !wwait_warp(&sm->never, 0, sm, p.status)) return;
     for (int j = 0; j < n; ++j) {
@@ -246,7 +247,8 @@ __device__ __forceinline__ void softmax_wide(SmemW* sm, const WideParams& p, uin
       l += rs;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);        // one arrival per warp (its stores are done)
     }
     const uint32_t n_commits = static_cast<uint32_t>(n) + (lin ? 1u : 0u);
     if (!wwait_warp(pv_done, (pv_phase + n_commits - 1) & 1u, sm, p.status)) return;
@@ -349,7 +351,7 @@ __global__ void __launch_bounds__(NTW, 1)
       mbar_init(&sm->q_full[s], 1);
       mbar_init(&sm->q_empty[s], 1);
       mbar_init(&sm->s_full[s], 1);
-      mbar_init(&sm->p_full[s], 256);
+      mbar_init(&sm->p_full[s], 8);             // one arrival per softmax warp of the slot
       mbar_init(&sm->pv_done[s], 1);
       mbar_init(&sm->ex1[s], 256);
       mbar_init(&sm->ex2[s], 256);
