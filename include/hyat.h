@@ -255,6 +255,17 @@ HYAT_API hyat_status hyat_stream_plan(const hyat_config* cfg, int32_t step, int3
 HYAT_API hyat_status hyat_stream_get_layout(hyat_handle h, int32_t* work, size_t work_cap, int32_t* entries,
                                    size_t entries_cap, int32_t* info, size_t info_len, int64_t* counts);
 
+/* Test hook: the persistent attention kernel's pair list as the last forward or streaming
+ * call left it, copied to the host (synchronises the device). 4 int32 per pair {item0,
+ * item1, shared, split}, items indexing the work list: pair k runs on CTA k mod
+ * min(n_pairs, SMs); item1 = -1 when the pair holds one query tile; shared = 1 when both
+ * query tiles have the same key-tile list (one K/V load serves both); split = 1 when the
+ * pair's two halves are item0's key tiles cut in two.
+ * In STREAM mode the prep kernel rewrites the list every step (largest key-tile count first,
+ * dealt in a serpentine) when the pairs are split pairs. *n_pairs always receives the count;
+ * a null `pairs` copies nothing; HYAT_ERR_INVALID_ARG if cap < 4 * n_pairs. */
+HYAT_API hyat_status hyat_get_pairs(hyat_handle h, int32_t* pairs, size_t cap, int64_t* n_pairs);
+
 /* Stream state (S, z, KV ring, step, and whether the current chunk's fold
  * has run) to / from a host buffer: a 48-byte header, then S, z as fp32
  * [B*H][d*d + d], then the K and V rings. The size is

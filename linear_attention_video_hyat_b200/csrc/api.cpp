@@ -120,6 +120,8 @@ struct hyat_ctx {
   // the zeroed status region
   bool single = false;
   bool wide = false;                 // two softmax warps per row (the default), with a redo list
+  bool order_on_device = false;      // streaming split pairs, ordered by the prep kernel each step
+  uint32_t* d_order_done = nullptr;  // the prep kernel's count of finished layout blocks
   int4* d_redo = nullptr;
   int32_t* d_redo_count = nullptr;
   uint32_t* d_redo_done = nullptr;
@@ -329,6 +331,7 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   }
   h->d_redo_count = reinterpret_cast<int32_t*>(ws + h->plan.status + 64);
   h->d_redo_done = reinterpret_cast<uint32_t*>(ws + h->plan.status + 128);
+  h->d_order_done = reinterpret_cast<uint32_t*>(ws + h->plan.status + 192);
 
   int dev = 0, major = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -362,7 +365,12 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
   if (cfg->mode == HYAT_MODE_STREAM) {
     const int32_t nqt = tiles(stream_chunk_tokens(*cfg));
     pairs = build_stream_pairs(h->BH, nqt);
-    if (prefer_split_pairs(pairs.size(), h->num_sms)) pairs = build_split_pairs(size_t(h->BH) * nqt);
+    if (prefer_split_pairs(pairs.size(), h->num_sms)) {
+      pairs = build_split_pairs(size_t(h->BH) * nqt);
+      // the key-tile counts change with every step's mask: the prep kernel deals the pairs
+      // out largest first (a table of one bin per possible count)
+      h->order_on_device = h->use_tc && nqt * stream_ring_slots(*cfg) + 1 <= kMaxStreamOrderBins;
+    }
   } else if (h->use_tc && (cfg->flags & HYAT_FLAG_SINGLE_TILE)) {
     pairs = build_single_items(h->lay.work, h->num_sms);
     h->single = true;
@@ -501,6 +509,9 @@ hyat_status enqueue_stream_call(hyat_handle h, const void* q, const void* k, con
   pa.H = c.H; pa.mask_heads = c.mask_heads; pa.nqt = nqt; pa.nkt = nqt * g.n_visible;
   pa.cap_entries = nqt * stream_ring_slots(c); pa.nwc = nwc;
   pa.n_sink_visible = g.n_sink_visible; pa.first_window_mod = g.first_window % nwc;
+  if (h->order_on_device) {
+    pa.pairs = h->d_pairs; pa.grid = std::min(h->n_pairs, h->num_sms); pa.done_counter = h->d_order_done;
+  }
   e = timed(h, K_PREP, s, [&] { return launch_stream_prep(pa, h->num_sms, s); });
   if (e != cudaSuccess) return cuda_fail(h, e, "stream prep kernel");
   const void* qa = c.rope_t_dims > 0 ? h->d_q_rot : q;
@@ -632,6 +643,18 @@ hyat_status hyat_stream_get_layout(hyat_handle h, int32_t* work, size_t work_cap
   if (e == cudaSuccess) e = cudaMemcpy(work, h->d_work, sizeof(WorkItem) * n_work, cudaMemcpyDeviceToHost);
   if (e == cudaSuccess) e = cudaMemcpy(entries, h->d_entries, sizeof(Entry) * n_ent, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(h, e, "layout copy");
+  return HYAT_OK;
+}
+
+hyat_status hyat_get_pairs(hyat_handle h, int32_t* pairs, size_t cap, int64_t* n_pairs) {
+  if (!h || !n_pairs) return HYAT_ERR_INVALID_ARG;
+  *n_pairs = h->n_pairs;
+  if (!pairs) return HYAT_OK;
+  if (cap < size_t(h->n_pairs) * 4) return fail(h, HYAT_ERR_INVALID_ARG, "pair buffer too small");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess && h->n_pairs > 0)
+    e = cudaMemcpy(pairs, h->d_pairs, sizeof(int4) * h->n_pairs, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "pair copy");
   return HYAT_OK;
 }
 

@@ -199,7 +199,15 @@ struct StreamPrepArgs {
   int32_t n_sink_visible;         // visible chunks 0..n_sink_visible-1 sit in slots nwc + c
   int32_t first_window_mod;       // first window chunk mod nwc: window chunk w sits in slot
                                   // (first_window_mod + w - n_sink_visible) % nwc
+  // Split-pair order (pairs != null): the last layout block to finish writes one split pair
+  // {item, item, 0, 1} per work item into pairs, largest key-tile count first, dealt to the
+  // attention's `grid` persistent CTAs in a serpentine (pair k runs on CTA k mod grid);
+  // done_counter counts finished layout blocks and is reset by the last one.
+  int4* pairs;
+  int32_t grid;
+  uint32_t* done_counter;
 };
+constexpr int32_t kMaxStreamOrderBins = 1024;   // split-pair ordering: key-tile counts 0..1023
 cudaError_t launch_stream_prep(StreamPrepArgs a, int num_sms, cudaStream_t s);
 
 }  // namespace hyat

@@ -40,6 +40,93 @@ __device__ __forceinline__ void turn_vector(uint4& v, int col, int half_t, const
   v = RopeLanes<T>::from_f32(f);
 }
 
+// Split pairs in the order the host gives bidirectional layouts (largest first, serpentine over
+// the persistent grid), from this step's key-tile counts. The layout blocks count themselves
+// done; the last one (it sees every work item, made visible by the others' fences before their
+// count) sorts the items by count, largest first, with a counting sort in shared memory. Equal
+// counts may land in any order: every pair is computed on its own, so the output does not
+// depend on it.
+__device__ __forceinline__ void order_split_pairs(const StreamPrepArgs& a) {
+  __shared__ int32_t bins[kMaxStreamOrderBins];
+  __shared__ int32_t is_last;
+  __threadfence();                                  // this thread's work item, before the count
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    is_last = atomicAdd(a.done_counter, 1u) == static_cast<uint32_t>(a.nb_layout - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const int n_items = a.BH * a.nqt;
+  const int nb = a.cap_entries + 1;               // counts 0 .. cap_entries
+  for (int b = threadIdx.x; b < nb; b += kPrepThreads) bins[b] = 0;
+  __syncthreads();
+  for (int it = threadIdx.x; it < n_items; it += kPrepThreads) {
+    const int n = __ldcg(&a.work[it].entry_end) - __ldcg(&a.work[it].entry_begin);
+    atomicAdd(&bins[n], 1);
+  }
+  __syncthreads();
+  // exclusive scan from the largest count down: bins[n] = number of items with a larger count
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x, per = (nb + 31) / 32;
+    const int hi = nb - 1 - lane * per;             // this lane's bins: hi, hi - 1, ..., > hi - per
+    int sum = 0;
+    for (int k = 0; k < per; ++k)
+      if (hi - k >= 0) sum += bins[hi - k];
+    int excl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, excl, off);
+      if (lane >= off) excl += t;
+    }
+    excl -= sum;
+    for (int k = 0; k < per; ++k) {
+      if (hi - k < 0) break;
+      const int c = bins[hi - k];
+      bins[hi - k] = excl;
+      excl += c;
+    }
+  }
+  __syncthreads();
+  for (int it = threadIdx.x; it < n_items; it += kPrepThreads) {
+    const int n = __ldcg(&a.work[it].entry_end) - __ldcg(&a.work[it].entry_begin);
+    const int k = atomicAdd(&bins[n], 1);           // sorted position, largest count first
+    const int row = k / a.grid, col = k % a.grid;
+    const int row_len = min(a.grid, n_items - row * a.grid);
+    const int c = (row & 1) ? row_len - 1 - col : col;
+    a.pairs[row * a.grid + c] = make_int4(it, it, 0, 1);
+  }
+  if (threadIdx.x == 0) *a.done_counter = 0u;       // for the next step
+}
+
+// One row of the step's tile mask (one warp per (bh, query tile)) compacted into its key-tile
+// list as ring rows; the diagonal tile of the newest chunk must be kept.
+__device__ __forceinline__ void layout_row(const StreamPrepArgs& a, int item) {
+  const int lane = threadIdx.x & 31;
+  const int bh = item / a.nqt, i = item % a.nqt;
+  const int hm = a.mask_heads == 1 ? 0 : bh % a.H;
+  const uint8_t* row = a.mask + (static_cast<int64_t>(hm) * a.nqt + i) * a.nkt;
+  const int64_t base = static_cast<int64_t>(item) * a.cap_entries;
+  int count = 0;
+  for (int kt0 = 0; kt0 < a.nkt; kt0 += 32) {
+    const int kt = kt0 + lane;
+    const bool keep = kt < a.nkt && row[kt] != 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int pos = count + __popc(bal & ((1u << lane) - 1u));
+      const int w = kt / a.nqt, t = kt % a.nqt;
+      const int slot = w < a.n_sink_visible ? a.nwc + w : (a.first_window_mod + w - a.n_sink_visible) % a.nwc;
+      a.entries[base + pos] = Entry{slot * a.L + t * kTile, min(kTile, a.L - t * kTile)};
+    }
+    count += __popc(bal);
+  }
+  if (lane == 0) {
+    if (row[a.nkt - a.nqt + i] == 0) atomicOr(a.status, kStatusBadMask);
+    a.work[item] = WorkItem{bh, i * kTile, min(kTile, a.L - i * kTile), 0, static_cast<int32_t>(base),
+                            static_cast<int32_t>(base + count), 0, 0};
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kPrepThreads) stream_prep_kernel(const StreamPrepArgs a) {
   extern __shared__ float2 cs_table[];            // [chunk frame][pair]: (cos, sin)
@@ -132,31 +219,9 @@ __global__ void __launch_bounds__(kPrepThreads) stream_prep_kernel(const StreamP
   b -= a.nb_kv + a.nb_q;
 
   // ---- layout: one warp per (bh, query tile)
-  const int lane = threadIdx.x & 31;
   const int item = b * (kPrepThreads / 32) + (threadIdx.x >> 5);
-  if (item >= a.BH * a.nqt) return;
-  const int bh = item / a.nqt, i = item % a.nqt;
-  const int hm = a.mask_heads == 1 ? 0 : bh % a.H;
-  const uint8_t* row = a.mask + (static_cast<int64_t>(hm) * a.nqt + i) * a.nkt;
-  const int64_t base = static_cast<int64_t>(item) * a.cap_entries;
-  int count = 0;
-  for (int kt0 = 0; kt0 < a.nkt; kt0 += 32) {
-    const int kt = kt0 + lane;
-    const bool keep = kt < a.nkt && row[kt] != 0;
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int pos = count + __popc(bal & ((1u << lane) - 1u));
-      const int w = kt / a.nqt, t = kt % a.nqt;
-      const int slot = w < a.n_sink_visible ? a.nwc + w : (a.first_window_mod + w - a.n_sink_visible) % a.nwc;
-      a.entries[base + pos] = Entry{slot * a.L + t * kTile, min(kTile, a.L - t * kTile)};
-    }
-    count += __popc(bal);
-  }
-  if (lane == 0) {
-    if (row[a.nkt - a.nqt + i] == 0) atomicOr(a.status, kStatusBadMask);
-    a.work[item] = WorkItem{bh, i * kTile, min(kTile, a.L - i * kTile), 0, static_cast<int32_t>(base),
-                            static_cast<int32_t>(base + count), 0, 0};
-  }
+  if (item < a.BH * a.nqt) layout_row(a, item);
+  if (a.pairs) order_split_pairs(a);                // every thread of the block takes part
 }
 
 int blocks_for(int64_t n, int cap) {
@@ -169,6 +234,7 @@ int blocks_for(int64_t n, int cap) {
 cudaError_t launch_stream_prep(StreamPrepArgs a, int num_sms, cudaStream_t s) {
   const int E = a.elem_bytes == 4 ? 4 : 8;
   if (a.d % E != 0 || (a.half_t > 0 && a.chunk_frames * a.half_t * 8 > 48 * 1024)) return cudaErrorInvalidValue;
+  if (a.pairs && (a.cap_entries + 1 > kMaxStreamOrderBins || a.grid < 1 || !a.done_counter)) return cudaErrorInvalidValue;
   const int64_t vecs = static_cast<int64_t>(a.L) * (a.d / E) * a.BH;
   a.nb_fold = a.partial ? blocks_for((static_cast<int64_t>(a.d) * a.d + a.d) / 4 * a.BH, 2 * num_sms) : 0;
   a.nb_kv = blocks_for((vecs + kPrepUnroll - 1) / kPrepUnroll, 8 * num_sms);

@@ -36,7 +36,7 @@ EXPORTED = (
     "hyat_stream_plan", "hyat_stream_state_bytes", "hyat_stream_get_state", "hyat_stream_set_state",
     "hyat_set_profiling", "hyat_kernel_times", "hyat_fwd_bidir_noalloc", "hyat_fwd_stream_denoise",
     "hyat_lvsa_mask", "hyat_rope_temporal", "hyat_fwd_stream_step_dev", "hyat_fwd_stream_step_graph",
-    "hyat_stream_get_layout",
+    "hyat_stream_get_layout", "hyat_get_pairs",
 )
 
 
@@ -74,6 +74,7 @@ def _load():
         "hyat_fwd_stream_step_dev": (ctypes.c_int, [P, P, P, P, P, P, P]),
         "hyat_fwd_stream_step_graph": (ctypes.c_int, [P, P, P, P, P, P, P]),
         "hyat_stream_get_layout": (ctypes.c_int, [P, P, S, P, S, P, S, ctypes.POINTER(I64)]),
+        "hyat_get_pairs": (ctypes.c_int, [P, P, S, ctypes.POINTER(I64)]),
         "hyat_sync": (ctypes.c_int, [P]),
         "hyat_destroy": (ctypes.c_int, [P]),
         "hyat_last_error": (ctypes.c_char_p, [P]),
@@ -296,6 +297,15 @@ class Hyat:
         _check(lib.hyat_stream_get_layout(self.handle, work.ctypes.data, work.size, ent.ctypes.data, ent.size,
                                           info.ctypes.data, info.size, counts), self.handle)
         return work, ent.reshape(n, ne // max(n, 1), 2), info, int(counts[2])
+
+    def pairs(self):
+        """The attention kernel's pair list as the last call left it: int32 [n_pairs, 4]
+        {item0, item1, shared, split}; pair k runs on CTA k mod min(n_pairs, SMs)."""
+        n = ctypes.c_int64()
+        _check(lib.hyat_get_pairs(self.handle, None, 0, ctypes.byref(n)), self.handle)
+        out = np.zeros((n.value, 4), np.int32)
+        _check(lib.hyat_get_pairs(self.handle, out.ctypes.data, out.size, ctypes.byref(n)), self.handle)
+        return out
 
     def stream_denoise(self, q, k, v, mask=None, out=None, stream=None):
         """A non-final call for the current chunk (one denoising step): attend with this

@@ -179,3 +179,44 @@ def test_stream_device_mask_without_diagonal_is_reported():
     h.stream_step(*_dev(q, k, v), mask=mask)
     h.sync()
     h.close()
+
+
+def test_stream_split_pairs_ordered_largest_first_on_device():
+    """With more query tiles than SMs' worth of pairs, the streaming attention runs split pairs,
+    and the prep kernel deals them out every step from that step's key-tile counts: each work
+    item once, and in dealing order (rows of min(n, SMs) pairs, every other row reversed) the
+    counts never grow. The outputs still match the oracle."""
+    w = wl.Workload("stream_order", "stream", 1, 60, 128, 100, 33, chunk_frames=3, window_frames=9,
+                    n_steps=7, seed=31)
+    h = hyat.Hyat(hyat.config_from_workload(w, mask_heads=w.H))
+    L, nwc = w.chunk_tokens, 3
+    G0 = torch.cuda.get_device_properties(0).multi_processor_count
+    kh, vh = [], []
+    for s in range(7):
+        q, k, v, mask = wl.gen_stream_step(w, s)
+        o = h.stream_step(*_dev(q, k, v), mask=mask)
+        kh.append(k.float().numpy())
+        vh.append(v.float().numpy())
+        work, _, _, _ = h.stream_layout()
+        pairs = h.pairs()
+        n = len(work)
+        assert len(pairs) == n and n > G0
+        assert sorted(pairs[:, 0].tolist()) == list(range(n))
+        assert (pairs[:, 1] == pairs[:, 0]).all() and (pairs[:, 2] == 0).all() and (pairs[:, 3] == 1).all()
+        G = min(n, G0)
+        counts = work[:, 5] - work[:, 4]
+        dealt = []
+        for k0 in range(n):
+            row, col = divmod(k0, G)
+            row_len = min(G, n - row * G)
+            dealt.append(counts[pairs[row * G + (row_len - 1 - col if row & 1 else col), 0]])
+        assert all(a >= b for a, b in zip(dealt, dealt[1:])), s
+        if s in (0, 6):
+            heads = [0, 1, 59]
+            got = f64(o.cpu())[:, heads]
+            want = oracle.stream_step_attention(f64(q)[:, heads], np.concatenate(kh, axis=2)[:, heads],
+                                                np.concatenate(vh, axis=2)[:, heads], s, L, nwc,
+                                                mask[heads], n_sink_chunks=0)
+            assert_parity("bf16", got, want, f"step {s}")
+    h.sync()
+    h.close()
