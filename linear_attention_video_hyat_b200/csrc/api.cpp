@@ -369,7 +369,8 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
       pairs = build_split_pairs(size_t(h->BH) * nqt);
       // the key-tile counts change with every step's mask: the prep kernel deals the pairs
       // out largest first (a table of one bin per possible count)
-      h->order_on_device = h->use_tc && nqt * stream_ring_slots(*cfg) + 1 <= kMaxStreamOrderBins;
+      h->order_on_device = h->use_tc && nqt * stream_ring_slots(*cfg) + 1 <= kMaxStreamOrderBins &&
+                           h->num_sms <= kMaxStreamOrderGrid && int64_t(h->BH) * nqt <= kMaxStreamOrderItems;
     }
   } else if (h->use_tc && (cfg->flags & HYAT_FLAG_SINGLE_TILE)) {
     pairs = build_single_items(h->lay.work, h->num_sms);
@@ -512,6 +513,10 @@ hyat_status enqueue_stream_call(hyat_handle h, const void* q, const void* k, con
   if (h->order_on_device) {
     pa.pairs = h->d_pairs; pa.grid = std::min(h->n_pairs, h->num_sms); pa.done_counter = h->d_order_done;
   }
+  // Ahead of the prep kernel: the fold's state kernel (a plain launch), or the previous call's
+  // attention kernels, which never trigger their dependents before they exit. Either way the
+  // previous attention has finished when the prep grid starts.
+  pa.layout_early = h->use_tc ? 1 : 0;
   e = timed(h, K_PREP, s, [&] { return launch_stream_prep(pa, h->num_sms, s); });
   if (e != cudaSuccess) return cuda_fail(h, e, "stream prep kernel");
   const void* qa = c.rope_t_dims > 0 ? h->d_q_rot : q;

@@ -13,7 +13,8 @@
 // Design for B200:
 //   * one persistent CTA per SM; a CTA owns a pair of 128-row query tiles
 //     ("slots"), so the softmax of one slot overlaps the MMAs of the other.
-//     Pairs are dealt largest first in a serpentine over the grid; when that
+//     Pairs are dealt largest first, a row of the grid at a time, each row to the
+//     CTAs least loaded so far (longest-processing-time first); when that
 //     would leave few waves, a "split pair" runs one query tile on both slots,
 //     each over half of its key tiles, and slot 0 merges the halves;
 //   * warp 8 issues TMA loads (Q tiles, K/V tiles, bf16 S_rest) into 128B-swizzled
@@ -448,6 +449,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
   pdl_wait();                // the linear states come from the kernels launched before this one
+  // No early trigger of dependents: the next streaming step's prep kernel relies on starting
+  // only once this kernel has exited, and then rewrites the work, entry and pair tables this
+  // kernel reads without a programmatic wait.
 
   if (warp >= 8) {
     // ------------------------------------------------------------ warpgroup 2: TMA + MMA

@@ -67,7 +67,8 @@ std::string build_layout(const hyat_config& c, const uint8_t* host_mask, Layout*
 // `shared` marks pairs whose key lists are identical (loaded once for both).
 std::vector<int4> build_pairs(const std::vector<WorkItem>& work);
 // Reorder pairs so that a persistent grid of `grid` CTAs, taking pair k on CTA k mod grid,
-// gets nearly equal work: largest pairs first, dealt out in a serpentine order.
+// gets nearly equal work: largest pairs first, each row of `grid` pairs dealt to the CTAs in
+// ascending order of the work they already hold.
 std::vector<int4> order_pairs_for_grid(const std::vector<int4>& pairs, const std::vector<WorkItem>& work,
                                        int32_t grid);
 std::vector<int4> build_stream_pairs(int32_t BH, int32_t nqt);
@@ -200,14 +201,20 @@ struct StreamPrepArgs {
   int32_t first_window_mod;       // first window chunk mod nwc: window chunk w sits in slot
                                   // (first_window_mod + w - n_sink_visible) % nwc
   // Split-pair order (pairs != null): the last layout block to finish writes one split pair
-  // {item, item, 0, 1} per work item into pairs, largest key-tile count first, dealt to the
-  // attention's `grid` persistent CTAs in a serpentine (pair k runs on CTA k mod grid);
-  // done_counter counts finished layout blocks and is reset by the last one.
+  // {item, item, 0, 1} per work item into pairs, largest key-tile count first, each row of
+  // `grid` pairs dealt to the attention's persistent CTAs least-loaded first (pair k runs on
+  // CTA k mod grid); done_counter counts finished layout blocks and is reset by the last one.
   int4* pairs;
   int32_t grid;
   uint32_t* done_counter;
+  // Nonzero: the kernel ahead of this one on the stream started only after the previous step's
+  // attention finished (a plain launch, or a programmatic launch whose primary triggers only at
+  // exit), so the layout blocks need not wait for it.
+  int32_t layout_early;
 };
 constexpr int32_t kMaxStreamOrderBins = 1024;   // split-pair ordering: key-tile counts 0..1023
+constexpr int32_t kMaxStreamOrderGrid = 1024;   // persistent grids of up to 1024 CTAs
+constexpr int32_t kMaxStreamOrderItems = 2048;  // and up to 2048 work items
 cudaError_t launch_stream_prep(StreamPrepArgs a, int num_sms, cudaStream_t s);
 
 }  // namespace hyat

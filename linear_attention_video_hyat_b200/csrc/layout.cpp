@@ -276,16 +276,36 @@ std::vector<int4> order_pairs_for_grid(const std::vector<int4>& pairs, const std
   std::vector<size_t> idx(pairs.size());
   for (size_t i = 0; i < idx.size(); ++i) idx[i] = i;
   std::stable_sort(idx.begin(), idx.end(), [&](size_t a, size_t b) { return cost[a] > cost[b]; });
-  // The kernel hands pair k to CTA k mod grid. Placing the pairs largest first in rows of
-  // `grid`, with every other row reversed, deals them out in a serpentine order.
-  std::vector<int4> out(pairs.size());
-  for (size_t k = 0; k < idx.size(); ++k) {
-    const size_t row = k / grid, col = k % grid;
-    const size_t row_len = std::min<size_t>(grid, idx.size() - row * grid);
-    const size_t c = (row & 1) ? row_len - 1 - col : col;
-    out[row * grid + c] = pairs[idx[k]];
+  // The kernel hands pair k to CTA k mod grid, so the list is rows of `grid` pairs, one per
+  // CTA, largest first. Two ways of placing each row's pairs are weighed, and the one whose
+  // busiest CTA holds less work wins (ties: the first):
+  //   * serpentine: left to right in even rows, right to left in odd rows;
+  //   * least loaded first: the row's pairs, largest first, to the CTAs in ascending order of
+  //     the work they already hold (ties: lower CTA), a longest-processing-time rule.
+  // Neither wins everywhere: with a few distinct costs the serpentine balances better, with
+  // widely spread costs the second.
+  const size_t n = idx.size();
+  std::vector<int4> serp(n), lpt(n);
+  std::vector<int64_t> load_s(grid, 0), load_l(grid, 0);
+  std::vector<int32_t> by_load(grid);
+  for (size_t r0 = 0, r = 0; r0 < n; r0 += grid, ++r) {
+    const size_t len = std::min<size_t>(grid, n - r0);   // a partial row: CTAs 0 .. len - 1
+    for (size_t j = 0; j < len; ++j) {
+      const size_t c = (r & 1) ? len - 1 - j : j;
+      serp[r0 + c] = pairs[idx[r0 + j]];
+      load_s[c] += cost[idx[r0 + j]];
+    }
+    for (size_t c = 0; c < len; ++c) by_load[c] = static_cast<int32_t>(c);
+    std::stable_sort(by_load.begin(), by_load.begin() + len, [&](int32_t a, int32_t b) { return load_l[a] < load_l[b]; });
+    for (size_t j = 0; j < len; ++j) {
+      const int32_t c = by_load[j];
+      lpt[r0 + c] = pairs[idx[r0 + j]];
+      load_l[c] += cost[idx[r0 + j]];
+    }
   }
-  return out;
+  const int64_t max_s = *std::max_element(load_s.begin(), load_s.end());
+  const int64_t max_l = *std::max_element(load_l.begin(), load_l.end());
+  return max_l < max_s ? lpt : serp;
 }
 
 std::vector<int4> build_split_pairs(size_t n_items) {

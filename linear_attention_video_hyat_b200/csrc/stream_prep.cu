@@ -11,10 +11,11 @@
 //   * Q rotation (fused RoPE only): Q turned into a workspace copy that the attention reads;
 //   * layout: one warp per (b, h, query tile) compacts its row of the step's tile mask into
 //     the key-tile list (ring rows), and checks that the diagonal tile of the newest chunk is
-//     kept.
-// The kernel streams its bytes once (HBM-bound); it waits for the fold's partial states (and
-// for the fold to have read the ring slot it overwrites) with a programmatic-launch wait, and
-// lets the attention kernel start its prologue early.
+//     kept; with split pairs, the last layout block to finish deals the pairs out to the
+//     attention's persistent CTAs from this step's key-tile counts.
+// The kernel streams its bytes once (HBM-bound); its copy blocks wait for the fold's partial
+// states (and for the fold to have read the ring slot they overwrite) with a programmatic-launch
+// wait, and it lets the attention kernel start its prologue early.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -40,31 +41,91 @@ __device__ __forceinline__ void turn_vector(uint4& v, int col, int half_t, const
   v = RopeLanes<T>::from_f32(f);
 }
 
-// Split pairs in the order the host gives bidirectional layouts (largest first, serpentine over
-// the persistent grid), from this step's key-tile counts. The layout blocks count themselves
-// done; the last one (it sees every work item, made visible by the others' fences before their
-// count) sorts the items by count, largest first, with a counting sort in shared memory. Equal
-// counts may land in any order: every pair is computed on its own, so the output does not
+// Split pairs dealt out from this step's key-tile counts, the way the host deals the pairs of
+// the bidirectional layouts. Largest count first, the list is rows of `grid` pairs (pair
+// r * grid + c runs on CTA c); two ways of placing each row's pairs are weighed, and the one
+// whose busiest CTA holds less work wins (ties: the first):
+//   * serpentine: left to right in even rows, right to left in odd rows;
+//   * least loaded first: each row's pairs, largest first, to the CTAs in ascending order of
+//     the work they already hold (longest-processing-time first, a row at a time).
+// A pair's work is its key tiles plus one for its set-up. The layout blocks count themselves
+// done; the last one (it sees every work item: each thread fences its writes before the count)
+// sorts the items with a counting sort in shared memory and deals the rows there, so that the
+// only global traffic is one read of the counts and one write of the list. Items of equal
+// count may land in any order: every pair is computed on its own, so the output does not
 // depend on it.
+struct OrderSmem {
+  int32_t bins[kMaxStreamOrderBins];    // histogram of counts, then first sorted position
+  int32_t sorted[kMaxStreamOrderItems]; // count << 20 | item, largest count first
+  int32_t load[kMaxStreamOrderGrid + 4];
+  int32_t dealt[kMaxStreamOrderItems];  // least-loaded-first: sorted position of each pair
+  int32_t is_last, serp_max;
+};
+
+__device__ __forceinline__ int sorted_cost(const OrderSmem& o, int k) { return (o.sorted[k] >> 20) + 1; }
+
+// Longest-processing-time dealing of the rows: dealt[r0 + c] = sorted position that goes to CTA
+// c in the row at r0. Returns the busiest CTA's work.
+__device__ __forceinline__ int deal_least_loaded(OrderSmem& o, int n_items, int grid) {
+  constexpr int kPer = (kMaxStreamOrderGrid + kPrepThreads - 1) / kPrepThreads;
+  for (int c = threadIdx.x; c < grid + 4; c += kPrepThreads) o.load[c] = 0;
+  __syncthreads();
+  for (int r0 = 0; r0 < n_items; r0 += grid) {
+    const int len = min(grid, n_items - r0);        // a partial last row: CTAs 0 .. len - 1
+    int add[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int c = threadIdx.x + u * kPrepThreads;
+      add[u] = 0;
+      if (c >= len) continue;
+      const int lc = o.load[c];
+      int rank = 0;                                 // CTAs holding less work (ties: lower index)
+      for (int c2 = 0; c2 < len; c2 += 4) {        // reads up to load[len + 2] < load[grid + 4]
+        const int4 l4 = *reinterpret_cast<const int4*>(&o.load[c2]);
+        rank += (c2 < len) & ((l4.x < lc) | ((l4.x == lc) & (c2 < c)));
+        rank += (c2 + 1 < len) & ((l4.y < lc) | ((l4.y == lc) & (c2 + 1 < c)));
+        rank += (c2 + 2 < len) & ((l4.z < lc) | ((l4.z == lc) & (c2 + 2 < c)));
+        rank += (c2 + 3 < len) & ((l4.w < lc) | ((l4.w == lc) & (c2 + 3 < c)));
+      }
+      o.dealt[r0 + c] = r0 + rank;
+      add[u] = sorted_cost(o, r0 + rank);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int c = threadIdx.x + u * kPrepThreads;
+      if (c < len) o.load[c] += add[u];
+    }
+    __syncthreads();
+  }
+  int mx = 0;
+  for (int c = 0; c < grid; ++c) mx = max(mx, o.load[c]);
+  return mx;
+}
+
 __device__ __forceinline__ void order_split_pairs(const StreamPrepArgs& a) {
-  __shared__ int32_t bins[kMaxStreamOrderBins];
-  __shared__ int32_t is_last;
+  __shared__ __align__(16) OrderSmem o;
   __threadfence();                                  // this thread's work item, before the count
   __syncthreads();
-  if (threadIdx.x == 0) {
-    is_last = atomicAdd(a.done_counter, 1u) == static_cast<uint32_t>(a.nb_layout - 1);
-  }
+  if (threadIdx.x == 0) o.is_last = atomicAdd(a.done_counter, 1u) == static_cast<uint32_t>(a.nb_layout - 1);
   __syncthreads();
-  if (!is_last) return;
+  if (!o.is_last) return;
   __threadfence();
-  const int n_items = a.BH * a.nqt;
-  const int nb = a.cap_entries + 1;               // counts 0 .. cap_entries
-  for (int b = threadIdx.x; b < nb; b += kPrepThreads) bins[b] = 0;
+  const int n_items = a.BH * a.nqt, grid = a.grid;
+  const int nb = a.cap_entries + 1;                 // counts 0 .. cap_entries
+  for (int b = threadIdx.x; b < nb; b += kPrepThreads) o.bins[b] = 0;
+  if (threadIdx.x == 0) o.serp_max = 0;
   __syncthreads();
-  for (int it = threadIdx.x; it < n_items; it += kPrepThreads) {
-    const int n = __ldcg(&a.work[it].entry_end) - __ldcg(&a.work[it].entry_begin);
-    atomicAdd(&bins[n], 1);
+  constexpr int kItemsPer = kMaxStreamOrderItems / kPrepThreads;
+  int cnt[kItemsPer];
+#pragma unroll
+  for (int u = 0; u < kItemsPer; ++u) {             // every count read in one round trip
+    const int it = threadIdx.x + u * kPrepThreads;
+    cnt[u] = it < n_items ? __ldcg(&a.work[it].entry_end) - __ldcg(&a.work[it].entry_begin) : -1;
   }
+#pragma unroll
+  for (int u = 0; u < kItemsPer; ++u)
+    if (cnt[u] >= 0) atomicAdd(&o.bins[cnt[u]], 1);
   __syncthreads();
   // exclusive scan from the largest count down: bins[n] = number of items with a larger count
   if (threadIdx.x < 32) {
@@ -72,7 +133,7 @@ __device__ __forceinline__ void order_split_pairs(const StreamPrepArgs& a) {
     const int hi = nb - 1 - lane * per;             // this lane's bins: hi, hi - 1, ..., > hi - per
     int sum = 0;
     for (int k = 0; k < per; ++k)
-      if (hi - k >= 0) sum += bins[hi - k];
+      if (hi - k >= 0) sum += o.bins[hi - k];
     int excl = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -82,19 +143,38 @@ __device__ __forceinline__ void order_split_pairs(const StreamPrepArgs& a) {
     excl -= sum;
     for (int k = 0; k < per; ++k) {
       if (hi - k < 0) break;
-      const int c = bins[hi - k];
-      bins[hi - k] = excl;
+      const int c = o.bins[hi - k];
+      o.bins[hi - k] = excl;
       excl += c;
     }
   }
   __syncthreads();
-  for (int it = threadIdx.x; it < n_items; it += kPrepThreads) {
-    const int n = __ldcg(&a.work[it].entry_end) - __ldcg(&a.work[it].entry_begin);
-    const int k = atomicAdd(&bins[n], 1);           // sorted position, largest count first
-    const int row = k / a.grid, col = k % a.grid;
-    const int row_len = min(a.grid, n_items - row * a.grid);
-    const int c = (row & 1) ? row_len - 1 - col : col;
-    a.pairs[row * a.grid + c] = make_int4(it, it, 0, 1);
+#pragma unroll
+  for (int u = 0; u < kItemsPer; ++u) {
+    const int it = threadIdx.x + u * kPrepThreads;
+    if (cnt[u] >= 0) o.sorted[atomicAdd(&o.bins[cnt[u]], 1)] = (cnt[u] << 20) | it;
+  }
+  __syncthreads();
+  // the serpentine's busiest CTA
+  for (int c = threadIdx.x; c < grid; c += kPrepThreads) {
+    int l = 0;
+    for (int r0 = 0, r = 0; r0 < n_items; r0 += grid, ++r) {
+      const int len = min(grid, n_items - r0);
+      if (c < len) l += sorted_cost(o, r0 + ((r & 1) ? len - 1 - c : c));
+    }
+    atomicMax(&o.serp_max, l);
+  }
+  const bool lpt = deal_least_loaded(o, n_items, grid) < o.serp_max;
+  for (int k = threadIdx.x; k < n_items; k += kPrepThreads) {
+    int src;
+    if (lpt) {
+      src = o.dealt[k];
+    } else {
+      const int r = k / grid, r0 = r * grid, len = min(grid, n_items - r0), c = k - r0;
+      src = r0 + ((r & 1) ? len - 1 - c : c);
+    }
+    const int it = o.sorted[src] & 0xfffff;
+    a.pairs[k] = make_int4(it, it, 0, 1);
   }
   if (threadIdx.x == 0) *a.done_counter = 0u;       // for the next step
 }
@@ -130,12 +210,29 @@ __device__ __forceinline__ void layout_row(const StreamPrepArgs& a, int item) {
 template <typename T>
 __global__ void __launch_bounds__(kPrepThreads) stream_prep_kernel(const StreamPrepArgs a) {
   extern __shared__ float2 cs_table[];            // [chunk frame][pair]: (cos, sin)
+  int b = blockIdx.x;
+
+  // ---- layout: one warp per (bh, query tile). These blocks come first in the grid. The
+  // layout depends on nothing the kernels before this one write: it reads the step's mask and
+  // writes the tables that the previous step's attention read. With `layout_early` the host
+  // states that this grid cannot start before that attention has finished (the kernel ahead of
+  // this one started only after it: a plain launch, or a programmatic launch whose primary
+  // triggers at exit), so these blocks skip the programmatic wait and run, pair ordering
+  // included, while the fold's state kernel still runs.
+  if (b < a.nb_layout) {
+    if (!a.layout_early) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int item = b * (kPrepThreads / 32) + (threadIdx.x >> 5);
+    if (item < a.BH * a.nqt) layout_row(a, item);
+    if (a.pairs) order_split_pairs(a);              // every thread of the block takes part
+    return;
+  }
+  b -= a.nb_layout;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int E = RopeLanes<T>::kElems;
   const int cols = a.d / E;                       // 16-byte vectors per row
   const int64_t row_vecs = static_cast<int64_t>(a.L) * cols;
-  int b = blockIdx.x;
 
   // ---- fold reduce: srest[bh] += sum_r partial[bh][r], r in order; bf16 copy of S
   if (b < a.nb_fold) {
@@ -216,12 +313,6 @@ __global__ void __launch_bounds__(kPrepThreads) stream_prep_kernel(const StreamP
     }
     return;
   }
-  b -= a.nb_kv + a.nb_q;
-
-  // ---- layout: one warp per (bh, query tile)
-  const int item = b * (kPrepThreads / 32) + (threadIdx.x >> 5);
-  if (item < a.BH * a.nqt) layout_row(a, item);
-  if (a.pairs) order_split_pairs(a);                // every thread of the block takes part
 }
 
 int blocks_for(int64_t n, int cap) {
@@ -234,7 +325,8 @@ int blocks_for(int64_t n, int cap) {
 cudaError_t launch_stream_prep(StreamPrepArgs a, int num_sms, cudaStream_t s) {
   const int E = a.elem_bytes == 4 ? 4 : 8;
   if (a.d % E != 0 || (a.half_t > 0 && a.chunk_frames * a.half_t * 8 > 48 * 1024)) return cudaErrorInvalidValue;
-  if (a.pairs && (a.cap_entries + 1 > kMaxStreamOrderBins || a.grid < 1 || !a.done_counter)) return cudaErrorInvalidValue;
+  if (a.pairs && (a.cap_entries + 1 > kMaxStreamOrderBins || a.grid < 1 || a.grid > kMaxStreamOrderGrid ||
+                  a.BH * a.nqt > kMaxStreamOrderItems || !a.done_counter)) return cudaErrorInvalidValue;
   const int64_t vecs = static_cast<int64_t>(a.L) * (a.d / E) * a.BH;
   a.nb_fold = a.partial ? blocks_for((static_cast<int64_t>(a.d) * a.d + a.d) / 4 * a.BH, 2 * num_sms) : 0;
   a.nb_kv = blocks_for((vecs + kPrepUnroll - 1) / kPrepUnroll, 8 * num_sms);

@@ -181,11 +181,28 @@ def test_stream_device_mask_without_diagonal_is_reported():
     h.close()
 
 
+def _deal_max_loads(sorted_costs, G):
+    """Busiest CTA's work under the two ways of dealing rows of G pairs (serpentine; least
+    loaded first), for costs sorted largest first."""
+    n = len(sorted_costs)
+    ls, ll = np.zeros(G, np.int64), np.zeros(G, np.int64)
+    for r, r0 in enumerate(range(0, n, G)):
+        m = min(G, n - r0)
+        row = sorted_costs[r0:r0 + m]
+        ls[:m] += row[::-1] if r & 1 else row
+        by_load = sorted(range(m), key=lambda c: (ll[c], c))
+        for j, c in enumerate(by_load):
+            ll[c] += row[j]
+    return ls.max(), ll.max()
+
+
 def test_stream_split_pairs_ordered_largest_first_on_device():
     """With more query tiles than SMs' worth of pairs, the streaming attention runs split pairs,
     and the prep kernel deals them out every step from that step's key-tile counts: each work
-    item once, and in dealing order (rows of min(n, SMs) pairs, every other row reversed) the
-    counts never grow. The outputs still match the oracle."""
+    item once, in rows of G = min(n, SMs) pairs (pair r * G + c on CTA c) that hold the counts
+    largest first. Within a row the pairs follow whichever rule leaves the busiest CTA less work
+    (key tiles + 1 per pair): a serpentine, or the larger counts to the CTAs holding less work so
+    far. The outputs still match the oracle."""
     w = wl.Workload("stream_order", "stream", 1, 60, 128, 100, 33, chunk_frames=3, window_frames=9,
                     n_steps=7, seed=31)
     h = hyat.Hyat(hyat.config_from_workload(w, mask_heads=w.H))
@@ -204,13 +221,22 @@ def test_stream_split_pairs_ordered_largest_first_on_device():
         assert sorted(pairs[:, 0].tolist()) == list(range(n))
         assert (pairs[:, 1] == pairs[:, 0]).all() and (pairs[:, 2] == 0).all() and (pairs[:, 3] == 1).all()
         G = min(n, G0)
-        counts = work[:, 5] - work[:, 4]
-        dealt = []
-        for k0 in range(n):
-            row, col = divmod(k0, G)
-            row_len = min(G, n - row * G)
-            dealt.append(counts[pairs[row * G + (row_len - 1 - col if row & 1 else col), 0]])
-        assert all(a >= b for a, b in zip(dealt, dealt[1:])), s
+        counts = (work[:, 5] - work[:, 4]).astype(np.int64)
+        want_rows = np.sort(counts)[::-1]
+        serp_max, lpt_max = _deal_max_loads(want_rows + 1, G)
+        lpt = lpt_max < serp_max
+        load = np.zeros(G, np.int64)
+        for r, r0 in enumerate(range(0, n, G)):
+            m = min(G, n - r0)
+            got = counts[pairs[r0:r0 + m, 0]]
+            assert np.array_equal(np.sort(got)[::-1], want_rows[r0:r0 + m]), (s, r0)
+            if lpt:
+                dealt = got[sorted(range(m), key=lambda c: (load[c], c))]
+            else:
+                dealt = got[::-1] if r & 1 else got
+            assert all(a >= b for a, b in zip(dealt, dealt[1:])), (s, r0, lpt)
+            load[:m] += got + 1
+        assert load.max() == min(serp_max, lpt_max)
         if s in (0, 6):
             heads = [0, 1, 59]
             got = f64(o.cpu())[:, heads]
