@@ -159,9 +159,12 @@ void lvsa_tile_mask(int32_t n_frames, int32_t F, int32_t window_frames, int32_t 
     }
 }
 
-static void push_window_entries(int64_t k_lo, int64_t k_hi, std::vector<Entry>* e) {
+// The key tiles of [k_lo, k_hi), first key first, or last tile first when `descending`.
+static void push_window_entries(int64_t k_lo, int64_t k_hi, bool descending, std::vector<Entry>* e) {
+  const size_t first = e->size();
   for (int64_t k = k_lo; k < k_hi; k += kTile)
     e->push_back(Entry{static_cast<int32_t>(k), static_cast<int32_t>(std::min<int64_t>(kTile, k_hi - k))});
+  if (descending) std::reverse(e->begin() + static_cast<std::ptrdiff_t>(first), e->end());
 }
 
 std::string build_layout(const hyat_config& c, const uint8_t* host_mask, Layout* L) {
@@ -185,7 +188,12 @@ std::string build_layout(const hyat_config& c, const uint8_t* host_mask, Layout*
       for (int32_t f = 0; f < T; ++f)
         L->cm[static_cast<size_t>(ch) * T + f] = (f < lo || f >= hi) ? 1.0f : 0.0f;
       eb[ch] = static_cast<int32_t>(L->entries.size());
-      push_window_entries(static_cast<int64_t>(lo) * F, static_cast<int64_t>(hi) * F, &L->entries);
+      // Neighbouring windows share the halo frames: the end of one window is the start of the
+      // next. Odd chunks walk their window last tile first, so the CTAs of two neighbouring
+      // chunks, which run at the same time, reach the shared frames at the same time and the
+      // second read of those K, V tiles hits L2 instead of HBM. (The sum over keys does not
+      // depend on their order beyond rounding.)
+      push_window_entries(static_cast<int64_t>(lo) * F, static_cast<int64_t>(hi) * F, (ch & 1) != 0, &L->entries);
       ee[ch] = static_cast<int32_t>(L->entries.size());
     }
     for (int32_t bh = 0; bh < BH; ++bh)

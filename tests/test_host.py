@@ -28,7 +28,7 @@ def _window_rows_from_layout(work, ent, bh=0):
     for w in work:
         if w[0] != bh:
             continue
-        keys = np.concatenate([np.arange(e[0], e[0] + e[1]) for e in ent[w[4]:w[5]]]) \
+        keys = np.sort(np.concatenate([np.arange(e[0], e[0] + e[1]) for e in ent[w[4]:w[5]]])) \
             if w[5] > w[4] else np.zeros(0, np.int64)
         for r in range(w[1], w[1] + w[2]):
             assert r not in rows
@@ -53,6 +53,11 @@ def test_window_layout_matches_oracle(T, F, C, h):
     assert np.all((ent[:, 1] >= 1) & (ent[:, 1] <= 128))
     for w in work:
         assert (w[1] // F) // C == ((w[1] + w[2] - 1) // F) // C
+        # even chunks list their key tiles first key first, odd chunks last tile first, with
+        # no gap or overlap between consecutive tiles
+        starts = ent[w[4]:w[5], 0]
+        step = np.diff(starts) if w[3] % 2 == 0 else -np.diff(starts)
+        assert np.all(step == 128), (w, starts[:4])
 
 
 def test_window_layout_tile_counts_wan13b():
