@@ -107,6 +107,17 @@ typedef enum {
  * default is the fastest on B200, the others are kept for cross-checks and timing. */
 #define HYAT_FLAG_SINGLE_TILE 4u
 #define HYAT_FLAG_PAIR_ONE_WARP 8u
+/* Test hooks for branch-wise parity (WINDOW, BLOCKMASK and RADIAL; STREAM and the
+ * allocation-free call reject them). A query row's output is (N_soft + N_lin) / (D_soft +
+ * D_lin): the softmax branch over its window keys and the linear branch over the rest (ReHyAt
+ * abstract; Hybrid Forcing, Section 2.A). With unit-variance inputs the linear branch carries
+ * most of the weight, so the hybrid output alone says little about the softmax branch.
+ * HYAT_FLAG_TEST_SOFTMAX_BRANCH zeroes the linear state between the complement and the
+ * attention kernel: the call returns N_soft / D_soft. HYAT_FLAG_TEST_LINEAR_BRANCH empties
+ * every query tile's key list when the handle is created: the call returns N_lin / D_lin =
+ * phi(q) S_rest / phi(q) z_rest. At most one of the two may be set. */
+#define HYAT_FLAG_TEST_SOFTMAX_BRANCH 16u
+#define HYAT_FLAG_TEST_LINEAR_BRANCH 32u
 
 typedef struct {
   int32_t B, H, d;               /* d in {64, 128} */

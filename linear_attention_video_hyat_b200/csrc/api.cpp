@@ -354,6 +354,10 @@ hyat_status hyat_create(const hyat_config* cfg, void* workspace, size_t workspac
     h->fold_parts = (Lc + h->fold_part_len - 1) / h->fold_part_len;
   }
 
+  // test hook: every query tile without softmax keys, so a call returns the linear branch
+  if (cfg->flags & HYAT_FLAG_TEST_LINEAR_BRANCH)
+    for (WorkItem& w : h->lay.work) w.entry_end = w.entry_begin;
+
   // layout tables and zeroed state
   e = cudaMemset(ws, 0, h->plan.status + 256);
   if (e == cudaSuccess && !h->lay.work.empty())
@@ -461,6 +465,13 @@ hyat_status hyat_fwd_bidir(hyat_handle h, const void* q, const void* k, const vo
     e = timed(h, K_COMPLEMENT, s, [&] { return launch_complement(ca, s); });
   }
   if (e != cudaSuccess) return cuda_fail(h, e, "complement kernel");
+  if (h->cfg.flags & HYAT_FLAG_TEST_SOFTMAX_BRANCH) {
+    // test hook: no linear state, so the call returns the softmax branch alone
+    e = cudaMemsetAsync(h->d_srest, 0, sizeof(float) * size_t(h->BH) * L.nqg * h->E, s);
+    if (e == cudaSuccess && h->d_srest_bf16)
+      e = cudaMemsetAsync(h->d_srest_bf16, 0, 2 * size_t(h->BH) * L.nqg * h->cfg.d * h->cfg.d, s);
+    if (e != cudaSuccess) return cuda_fail(h, e, "branch test hook");
+  }
   return launch_attention(h, attn_args(h, q, k, v, o, h->plan.n_work, L.nqg), s);
 }
 

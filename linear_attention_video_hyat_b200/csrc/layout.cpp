@@ -81,6 +81,10 @@ std::string validate_config(const hyat_config& c) {
     default:
       return "unknown mode";
   }
+  const uint32_t branch = c.flags & (HYAT_FLAG_TEST_SOFTMAX_BRANCH | HYAT_FLAG_TEST_LINEAR_BRANCH);
+  if (branch == (HYAT_FLAG_TEST_SOFTMAX_BRANCH | HYAT_FLAG_TEST_LINEAR_BRANCH))
+    return "at most one of the branch test flags";
+  if (branch && c.mode == HYAT_MODE_STREAM) return "the branch test flags are for the bidirectional modes";
   if (c.rope_t_dims != 0) {
     if (c.mode != HYAT_MODE_STREAM) return "the fused temporal RoPE is a STREAM option";
     if (c.rope_t_dims < 0 || c.rope_t_dims > c.d || c.rope_t_dims % 2 != 0)

@@ -70,6 +70,7 @@ extern "C" HYAT_API hyat_status hyat_fwd_bidir_noalloc(const hyat_config* cfg, c
   if (!cfg || !q || !k || !v || !o) return HYAT_ERR_INVALID_ARG;
   if (!validate_config(*cfg).empty()) return HYAT_ERR_INVALID_ARG;
   if (cfg->mode != HYAT_MODE_WINDOW && cfg->mode != HYAT_MODE_RADIAL) return HYAT_ERR_INVALID_ARG;
+  if (cfg->flags & (HYAT_FLAG_TEST_SOFTMAX_BRANCH | HYAT_FLAG_TEST_LINEAR_BRANCH)) return HYAT_ERR_UNSUPPORTED;
   for (const void* p : {q, k, v, static_cast<const void*>(o)})
     if (reinterpret_cast<uintptr_t>(p) & 15u) return HYAT_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

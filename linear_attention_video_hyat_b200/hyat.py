@@ -24,6 +24,8 @@ FLAG_SIMT = 1
 FLAG_TEST_DEVICE_TIMEOUT = 2
 FLAG_SINGLE_TILE = 4
 FLAG_PAIR_ONE_WARP = 8
+FLAG_TEST_SOFTMAX_BRANCH = 16     # test hook: the call returns the softmax branch alone
+FLAG_TEST_LINEAR_BRANCH = 32      # test hook: the call returns the linear branch alone
 TILE = 128
 KERNEL_KINDS = ("state", "complement", "attention", "fold", "prep")
 

@@ -122,7 +122,10 @@ def test_stream_plan_eviction_indexing():
 
 @pytest.mark.parametrize("bad", [dict(d=96), dict(B=0), dict(tokens_per_frame=0), dict(mode=9),
                                  dict(mode="stream", window_frames=8), dict(mode="blockmask", mask_heads=3),
-                                 dict(dtype=7), dict(scale=-1.0), dict(phi=3), dict(phi=-1)])
+                                 dict(dtype=7), dict(scale=-1.0), dict(phi=3), dict(phi=-1),
+                                 dict(flags=hyat.FLAG_TEST_SOFTMAX_BRANCH | hyat.FLAG_TEST_LINEAR_BRANCH),
+                                 dict(mode="stream", flags=hyat.FLAG_TEST_SOFTMAX_BRANCH),
+                                 dict(mode="stream", flags=hyat.FLAG_TEST_LINEAR_BRANCH)])
 def test_invalid_configs_rejected(bad):
     kw = dict(mode="window", B=1, H=2, d=64, tokens_per_frame=64, n_frames=4, chunk_frames=1,
               window_frames=9)
@@ -131,6 +134,13 @@ def test_invalid_configs_rejected(bad):
         kw["chunk_frames"] = 3
     cfg = hyat.make_config(**kw)
     assert hyat.workspace_bytes(cfg) == 0
+
+
+@pytest.mark.parametrize("flags", [0, hyat.FLAG_TEST_SOFTMAX_BRANCH, hyat.FLAG_TEST_LINEAR_BRANCH])
+def test_branch_flags_accepted_in_bidirectional_modes(flags):
+    for mode in ("window", "radial"):
+        cfg = hyat.make_config(mode, 1, 2, 64, 64, 4, 1, 0, flags=flags)
+        assert hyat.workspace_bytes(cfg) > 0
 
 
 @pytest.mark.parametrize("rope,ok", [({"t_dims": 44, "cap": 21}, True), ({"t_dims": 128, "cap": 1, "base": 500.0}, True),
