@@ -524,8 +524,9 @@ hyat_status enqueue_stream_call(hyat_handle h, const void* q, const void* k, con
   if (h->order_on_device) {
     pa.pairs = h->d_pairs; pa.grid = std::min(h->n_pairs, h->num_sms); pa.done_counter = h->d_order_done;
   }
-  // Ahead of the prep kernel: the fold's state kernel (a plain launch), or the previous call's
-  // attention kernels, which never trigger their dependents before they exit. Either way the
+  // Ahead of the prep kernel: the fold's state kernel, or the previous call's attention
+  // kernels, which never trigger their dependents before they exit (so the fold, a
+  // programmatic launch behind them, starts only once they have exited). Either way the
   // previous attention has finished when the prep grid starts.
   pa.layout_early = h->use_tc ? 1 : 0;
   e = timed(h, K_PREP, s, [&] { return launch_stream_prep(pa, h->num_sms, s); });

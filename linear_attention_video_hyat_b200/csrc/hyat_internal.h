@@ -208,8 +208,8 @@ struct StreamPrepArgs {
   int32_t grid;
   uint32_t* done_counter;
   // Nonzero: the kernel ahead of this one on the stream started only after the previous step's
-  // attention finished (a plain launch, or a programmatic launch whose primary triggers only at
-  // exit), so the layout blocks need not wait for it.
+  // attention finished (a programmatic launch whose primary triggers only at exit), so the
+  // layout blocks need not wait for it.
   int32_t layout_early;
 };
 constexpr int32_t kMaxStreamOrderBins = 1024;   // split-pair ordering: key-tile counts 0..1023

@@ -268,6 +268,9 @@ __global__ void __launch_bounds__(ST_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
+  // Launched programmatically: the set-up above overlaps the end of the kernel before this one;
+  // K, V (and the ring slot a fold reads) are read, and any output written, only after its wait.
+  pdl_wait();
   pdl_launch_dependents();   // the complement kernel may begin launching; it waits for our results
 
   if (warp == ST_TMA_WARP) {
@@ -381,8 +384,7 @@ cudaError_t launch_seg_state_tc(const SegStateArgs& a, int num_sms, cudaStream_t
   p.out_lo = a.out_lo;
   p.phi = a.phi;
   const int grid = p.n_units < num_sms ? p.n_units : num_sms;
-  state_tc_kernel<<<grid, ST_THREADS, kStateSmemBytes, s>>>(mk, mv, p);
-  return cudaGetLastError();
+  return launch_pdl(state_tc_kernel, dim3(grid), dim3(ST_THREADS), kStateSmemBytes, s, mk, mv, p);
 }
 
 }  // namespace hyat

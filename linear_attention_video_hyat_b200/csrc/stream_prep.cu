@@ -216,9 +216,9 @@ __global__ void __launch_bounds__(kPrepThreads) stream_prep_kernel(const StreamP
   // layout depends on nothing the kernels before this one write: it reads the step's mask and
   // writes the tables that the previous step's attention read. With `layout_early` the host
   // states that this grid cannot start before that attention has finished (the kernel ahead of
-  // this one started only after it: a plain launch, or a programmatic launch whose primary
-  // triggers at exit), so these blocks skip the programmatic wait and run, pair ordering
-  // included, while the fold's state kernel still runs.
+  // this one started only after it: a programmatic launch whose primary triggers at exit), so
+  // these blocks skip the programmatic wait and run, pair ordering included, while the fold's
+  // state kernel still runs.
   if (b < a.nb_layout) {
     if (!a.layout_early) asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
