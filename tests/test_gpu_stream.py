@@ -246,3 +246,28 @@ def test_stream_split_pairs_ordered_largest_first_on_device():
             assert_parity("bf16", got, want, f"step {s}")
     h.sync()
     h.close()
+
+
+def test_stream_split_pairs_beyond_the_device_order_limit():
+    """A window of 28 chunks: a query tile may keep up to 37 x 28 = 1036 key tiles, more
+    counts than the prep kernel's ordering table holds (1024), so the split pairs keep their
+    list order; the steps still match the oracle."""
+    w = wl.Workload("stream_long_window", "stream", 1, 2, 128, 1560, 6, chunk_frames=3, window_frames=84,
+                    n_steps=2, seed=41)
+    h = hyat.Hyat(hyat.config_from_workload(w, mask_heads=w.H))
+    L, nwc = w.chunk_tokens, 28
+    kh, vh = [], []
+    for s in range(2):
+        q, k, v, mask = wl.gen_stream_step(w, s)
+        o = h.stream_step(*_dev(q, k, v), mask=mask)
+        kh.append(k.float().numpy())
+        vh.append(v.float().numpy())
+        pairs = h.pairs()
+        n = 2 * 37
+        assert len(pairs) == n and np.array_equal(pairs[:, 0], np.arange(n)) and (pairs[:, 3] == 1).all()
+        rows = np.unique(np.concatenate([np.arange(0, L, 61), [L - 1]]))
+        want = oracle.stream_step_attention(f64(q), np.concatenate(kh, axis=2), np.concatenate(vh, axis=2), s, L,
+                                            nwc, mask, rows=rows, n_sink_chunks=0)
+        assert_parity("bf16", f64(o.cpu())[:, :, rows], want, f"step {s}")
+    h.sync()
+    h.close()
