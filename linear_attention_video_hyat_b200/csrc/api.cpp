@@ -524,11 +524,12 @@ hyat_status enqueue_stream_call(hyat_handle h, const void* q, const void* k, con
   if (h->order_on_device) {
     pa.pairs = h->d_pairs; pa.grid = std::min(h->n_pairs, h->num_sms); pa.done_counter = h->d_order_done;
   }
-  // Ahead of the prep kernel: the fold's state kernel, or the previous call's attention
-  // kernels, which never trigger their dependents before they exit (so the fold, a
-  // programmatic launch behind them, starts only once they have exited). Either way the
-  // previous attention has finished when the prep grid starts.
-  pa.layout_early = h->use_tc ? 1 : 0;
+  // When this call folds, the kernel ahead of the prep kernel is the fold's state kernel,
+  // which triggers the prep grid only after its own programmatic wait: by then everything
+  // enqueued before this call (the previous step's attention, a kernel that wrote a device
+  // mask) has finished, so the prep kernel's layout blocks need not wait. Without a fold the
+  // kernel ahead could be anything the caller enqueued, so they wait.
+  pa.layout_early = (h->use_tc && fold) ? 1 : 0;
   e = timed(h, K_PREP, s, [&] { return launch_stream_prep(pa, h->num_sms, s); });
   if (e != cudaSuccess) return cuda_fail(h, e, "stream prep kernel");
   const void* qa = c.rope_t_dims > 0 ? h->d_q_rot : q;

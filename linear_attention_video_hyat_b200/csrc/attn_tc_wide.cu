@@ -376,9 +376,9 @@ __global__ void __launch_bounds__(NTW, 1)
   tc_fence_after();
   const uint32_t tmem = sm->tmem_base;
   pdl_wait();                // the linear states come from the kernels launched before this one
-  // No early trigger of dependents: the next streaming step's prep kernel relies on starting
-  // only once this kernel has exited, and then rewrites the work, entry and pair tables this
-  // kernel reads without a programmatic wait.
+  // No early trigger of dependents: the next streaming step's fold starts only once this
+  // kernel has exited, and the prep kernel behind the fold rewrites the work, entry and pair
+  // tables this kernel reads.
 
   if (warp == TMA_WARP) {
     if (lane == 0) {

@@ -207,9 +207,9 @@ struct StreamPrepArgs {
   int4* pairs;
   int32_t grid;
   uint32_t* done_counter;
-  // Nonzero: the kernel ahead of this one on the stream started only after the previous step's
-  // attention finished (a programmatic launch whose primary triggers only at exit), so the
-  // layout blocks need not wait for it.
+  // Nonzero: the kernel ahead of this one on the stream is the fold's state kernel, which lets
+  // this grid start only after its own programmatic wait (everything enqueued before the call
+  // has finished by then), so the layout blocks need not wait.
   int32_t layout_early;
 };
 constexpr int32_t kMaxStreamOrderBins = 1024;   // split-pair ordering: key-tile counts 0..1023

@@ -190,7 +190,7 @@ __device__ __forceinline__ void layout_row(const StreamPrepArgs& a, int item) {
   int count = 0;
   for (int kt0 = 0; kt0 < a.nkt; kt0 += 32) {
     const int kt = kt0 + lane;
-    const bool keep = kt < a.nkt && row[kt] != 0;
+    const bool keep = kt < a.nkt && __ldcg(row + kt) != 0;
     const unsigned bal = __ballot_sync(0xffffffffu, keep);
     if (keep) {
       const int pos = count + __popc(bal & ((1u << lane) - 1u));
@@ -201,7 +201,7 @@ __device__ __forceinline__ void layout_row(const StreamPrepArgs& a, int item) {
     count += __popc(bal);
   }
   if (lane == 0) {
-    if (row[a.nkt - a.nqt + i] == 0) atomicOr(a.status, kStatusBadMask);
+    if (__ldcg(row + (a.nkt - a.nqt + i)) == 0) atomicOr(a.status, kStatusBadMask);
     a.work[item] = WorkItem{bh, i * kTile, min(kTile, a.L - i * kTile), 0, static_cast<int32_t>(base),
                             static_cast<int32_t>(base + count), 0, 0};
   }
@@ -213,12 +213,12 @@ __global__ void __launch_bounds__(kPrepThreads) stream_prep_kernel(const StreamP
   int b = blockIdx.x;
 
   // ---- layout: one warp per (bh, query tile). These blocks come first in the grid. The
-  // layout depends on nothing the kernels before this one write: it reads the step's mask and
-  // writes the tables that the previous step's attention read. With `layout_early` the host
-  // states that this grid cannot start before that attention has finished (the kernel ahead of
-  // this one started only after it: a programmatic launch whose primary triggers at exit), so
-  // these blocks skip the programmatic wait and run, pair ordering included, while the fold's
-  // state kernel still runs.
+  // layout reads the step's mask and writes the tables that the previous step's attention
+  // read; the fold's state kernel writes neither. With `layout_early` the host states that the
+  // kernel ahead of this one is the fold, which lets this grid start only after its own
+  // programmatic wait, i.e. once everything enqueued before the call (that attention, a kernel
+  // that wrote the mask) has finished; so these blocks skip the wait and run, pair ordering
+  // included, while the fold still runs. They read the mask past L1 (`__ldcg`).
   if (b < a.nb_layout) {
     if (!a.layout_early) asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
