@@ -43,6 +43,11 @@ KERNEL_SOURCES = ["linear_attention_video_hyat_b200/csrc/attn_tc_wide.cu", "line
 ROPE = {"t_dims": 44, "cap": 21, "base": 10000.0}
 
 
+
+# Idle time before the per-launch timing pass: the 1000 W power limit lowers the SM clock after
+# the timed pass's load; a second of idle lets the kernel pass run at the timed pass's clocks.
+KERNEL_PASS_IDLE_S = 1.0
+
 def l2_note(io_bytes):
     """How the timed region stands to the 126 MB L2: the full-size layers' inputs exceed it."""
     mb = io_bytes / 1e6
@@ -461,6 +466,7 @@ def bench_stream(a, w, rank, world, local):
     h.sync()
     ms = max_over_ranks(t0.elapsed_time(t1) / a.steps, dev)
     first += a.steps
+    time.sleep(KERNEL_PASS_IDLE_S)
     h.set_profiling(True)        # per-launch events (graph replay is off while profiling)
     h.kernel_times()
     with ClockSampler(local) as clk2:
@@ -660,7 +666,10 @@ def main():
     h.sync()
     ms = t0.elapsed_time(t1) / a.steps
     # Pass 2: K more steps with CUDA events around every launch (library-side), for the
-    # per-kernel durations of the roofline.
+    # per-kernel durations of the roofline. It starts after an idle second, so that it runs at
+    # the clocks of pass 1 instead of those the power limit sets after pass 1's load (both
+    # passes' clocks are in the line).
+    time.sleep(KERNEL_PASS_IDLE_S)
     h.set_profiling(True)
     h.kernel_times()
     with ClockSampler(local) as clk2:
