@@ -20,6 +20,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -47,6 +48,19 @@ ROPE = {"t_dims": 44, "cap": 21, "base": 10000.0}
 # Idle time before the per-launch timing pass: the 1000 W power limit lowers the SM clock after
 # the timed pass's load; a second of idle lets the kernel pass run at the timed pass's clocks.
 KERNEL_PASS_IDLE_S = 1.0
+
+
+
+def kernel_source_digest() -> str:
+    """sha256 of the attention kernels' sources with comments and runs of blank space removed:
+    the DRAM traffic record stays valid across edits of comments only, and lapses with any
+    change to the code."""
+    def code(path):
+        t = open(os.path.join(ROOT, path), encoding="utf-8").read()
+        t = re.sub(r"/\*.*?\*/", " ", t, flags=re.S)
+        t = re.sub(r"//[^\n]*", " ", t)
+        return re.sub(r"\s+", " ", t).strip().encode()
+    return hashlib.sha256(b"".join(code(f) for f in KERNEL_SOURCES)).hexdigest()
 
 def l2_note(io_bytes):
     """How the timed region stands to the 126 MB L2: the full-size layers' inputs exceed it."""
@@ -691,7 +705,7 @@ def main():
     tpath = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if os.path.exists(tpath):
         t = json.load(open(tpath))
-        sha = hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read() for f in KERNEL_SOURCES)).hexdigest()
+        sha = kernel_source_digest()
         if t.get("source_sha256") == sha and t.get("workload") == w.name and t.get("schedule", "pair") == a.schedule:
             traffic = t.get("dram_bytes_per_launch")
     roofline = {"bound": "tensor", "kernel": "attention", "achieved": achieved,
