@@ -22,6 +22,20 @@ def test_library_exports_every_declared_symbol():
     assert sorted(hyat.EXPORTED) == declared
 
 
+def test_binding_constants_match_the_header():
+    """Every HYAT_FLAG_*, status and enum value the binding names has the header's value."""
+    header = open(os.path.join(ROOT, "include", "hyat.h")).read()
+    flags = dict(re.findall(r"#define HYAT_FLAG_(\w+) (\d+)u", header))
+    assert len(flags) >= 6
+    for name, val in flags.items():
+        assert getattr(hyat, "FLAG_" + name) == int(val), name
+    enums = dict((n, int(v)) for n, v in re.findall(r"\bHYAT_(\w+) = (\d+)", header))
+    for name in ("OK", "ERR_INVALID_ARG", "ERR_UNSUPPORTED", "ERR_CUDA", "ERR_DEVICE_TIMEOUT", "ERR_STATE",
+                 "F32", "BF16", "MODE_WINDOW", "MODE_BLOCKMASK", "MODE_RADIAL", "MODE_STREAM"):
+        if name in enums:
+            assert getattr(hyat, name) == enums[name], name
+
+
 def _window_rows_from_layout(work, ent, bh=0):
     """Map query row -> sorted array of softmax keys, from the C++ layout."""
     rows = {}
