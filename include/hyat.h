@@ -272,10 +272,14 @@ HYAT_API hyat_status hyat_stream_get_layout(hyat_handle h, int32_t* work, size_t
  * min(n_pairs, SMs); item1 = -1 when the pair holds one query tile; shared = 1 when both
  * query tiles have the same key-tile list (one K/V load serves both); split = 1 when the
  * pair's two halves are item0's key tiles cut in two.
- * In STREAM mode the prep kernel rewrites the list every step when the pairs are split pairs:
- * largest key-tile count first, each row of min(n_pairs, SMs) pairs dealt to the CTAs in
- * ascending order of the key tiles (plus one per pair) they already hold. *n_pairs always receives the count;
- * a null `pairs` copies nothing; HYAT_ERR_INVALID_ARG if cap < 4 * n_pairs. */
+ * The list holds the pairs largest first (key tiles of both items + 2), in rows of
+ * min(n_pairs, SMs) pairs, each row placed in a serpentine or least loaded first (the row's
+ * pairs to the CTAs holding the least work so far), whichever leaves the busiest CTA less
+ * work. In STREAM mode with split pairs the prep kernel rewrites the list every step by the
+ * same rule from that step's key-tile counts (cost: key tiles + 1), as long as the step has at
+ * most 2048 query tiles, 1023 key tiles per query tile and 1024 CTAs; otherwise the list keeps
+ * its creation order. *n_pairs always receives the count; a null `pairs` copies nothing;
+ * HYAT_ERR_INVALID_ARG if cap < 4 * n_pairs. */
 HYAT_API hyat_status hyat_get_pairs(hyat_handle h, int32_t* pairs, size_t cap, int64_t* n_pairs);
 
 /* Stream state (S, z, KV ring, step, and whether the current chunk's fold
